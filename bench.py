@@ -1,0 +1,414 @@
+"""Benchmark of one verification step on B200 (see the JSON contract below).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step = dual-view attention (one layer, with d_in/d_out) + vocabulary
+verification + seed selection + decisions on the workload's whole batch,
+replayed from three CUDA graphs. Inputs are synthetic (seeded), shaped like
+the LLaDA-8B L=512 verification step by default.
+
+Rank 0 prints one JSON line:
+  value     whole-job verify steps/s, device-timed (CUDA events, L2 flushed
+            between steps, max over ranks); positions_per_s = value * B * R
+  e2e       the same step through the public API with pinned HOST buffers:
+            host->device copy of every input and device->host copy of the
+            decisions inside each timed step
+  roofline  the dominant kernel (the vocabulary pass: HBM-bound) against the
+            measured HBM copy bandwidth; attention is reported beside it
+            against the measured dense bf16 tensor peak
+  cpu_baseline  the fp64 CPU oracle on a bounded sample (rank 0, N = 1 only)
+Under torchrun (N > 1) each rank runs its own batch (weak scaling, no
+collective on the data path; the only collectives are the timing barrier and
+max-reduce).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from speculative_verification_cover_b200 import workloads as W  # noqa: E402
+
+METRIC = "verify steps/s & positions/s at L=512 LLaDA-8B shape; % HBM/TC roofline"
+FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=1000)
+    p.add_argument("--warmup", type=int, default=50)
+    p.add_argument("--workload", default=W.LLADA8B_L512.name)
+    p.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def spec_by_name(name):
+    for s in W.WORKLOADS:
+        if s.name == name or s.name.startswith(name):
+            return s
+    raise SystemExit(f"unknown workload {name}")
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            m = json.load(f)
+        return m["hbm_gbs"], m["bf16_tflops"], m.get("bf16_tflops_sustained"), "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+# ----------------------------------------------------------------------------- dist
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def shard_seed(spec, rank):
+    """Each rank verifies its own batch of the workload (independent sequences)."""
+    return W.default_seed(spec) + 7919 * rank
+
+
+def max_over_ranks(values, world):
+    t = torch.tensor(values, dtype=torch.float64,
+                     device="cuda" if torch.cuda.is_available() else "cpu")
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Polls NVML during the timed region (SM clock, max clock, throttle reasons)."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # NVML missing: report it instead of guessing
+            self.err = str(e)
+
+    def _poll(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit and bit != 0x1:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._poll, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": self.err}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- roofline data
+def algorithmic(spec):
+    esize = 4 if spec.dtype == "f32" else 2
+    verify_bytes = 2 * spec.B * spec.R * spec.V * esize
+    masked = spec.masked if not spec.tree else spec.block - 1
+    attn_flops = 4 * spec.B * spec.Hq * spec.L ** 2 * spec.d
+    pass2_flops = 2 * spec.B * spec.Hq * masked * spec.L * spec.d
+    return verify_bytes, attn_flops, pass2_flops
+
+
+def recorded_traffic(kernel_file, workload_name):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
+    current source of the kernel (its sha256 is recorded beside the figure)."""
+    src = os.path.join(ROOT, "speculative_verification_cover_b200", "csrc", kernel_file)
+    summ = os.path.join(ROOT, "profiles", "verify_logits_%s.md" % workload_name.split("_")[0])
+    if not (os.path.exists(src) and os.path.exists(summ)):
+        return None
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    rec = {}
+    for line in open(summ):
+        if line.startswith("traffic_bytes_per_launch:"):
+            rec["bytes"] = float(line.split(":", 1)[1])
+        if line.startswith("source_sha256_16:"):
+            rec["sha"] = line.split(":", 1)[1].strip()
+    if rec.get("sha") == h and "bytes" in rec:
+        return rec["bytes"]
+    return None
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def oracle_step(x, spec, b, head_stride=1, row_stride=1, seed=2024, step_index=1):
+    """One verification step of sequence b on the CPU oracle (optionally a sample:
+    every head_stride-th head and every row_stride-th verified row). Returns seconds
+    per full step, extrapolated from the sample."""
+    from oracle import attention as OA
+    from oracle import decide as OD
+    from oracle import seeds as OS
+    from oracle import vocab as OV
+    f64 = lambda t: t.detach().float().cpu().numpy().astype(np.float64)
+    q, kc, vc, kp, vp = (f64(x[k][b]) for k in ("q", "k_cur", "v_cur", "k_prev", "v_prev"))
+    seeds = x["is_seed"][b].cpu().numpy()
+    masked = x["is_masked"][b].cpu().numpy().astype(bool)
+    heads = np.arange(0, spec.Hq, head_stride)
+    rows = np.arange(0, spec.R, row_stride)
+    lt = f64(x["logits_t"][b][torch.as_tensor(rows, device=x["logits_t"].device)])
+    lm = f64(x["logits_d"][b][torch.as_tensor(rows, device=x["logits_d"].device)])
+    t0 = time.perf_counter()
+    out, lse, A = OA.dualview_attention(q, kc, vc, kp, vp, seeds, heads=heads)
+    d_in = OA.d_in(A[:, masked, :], len(heads))
+    d_out = OA.d_out(A, x["is_new"][b].cpu().numpy(), len(heads))
+    t1 = time.perf_counter()
+    st = OV.verify_rows(lt, lm, spec.temperature, seed, step_index, b, rows + spec.pos_offset)
+    t2 = time.perf_counter()
+    u = np.zeros(spec.L)
+    u[spec.pos_offset + rows] = st["entropy_t"]
+    score = OS.stability_score(u, d_in, d_out, x["eligible"][b].cpu().numpy())
+    OS.select(score, max(spec.k, 1))
+    full = {k: np.zeros(spec.R, dtype=v.dtype) for k, v in st.items()}
+    for k, v in st.items():
+        full[k][rows] = v
+    OD.decide(spec.policy, x["tokens"][b].cpu().numpy(), seeds, x["eligible"][b].cpu().numpy(),
+              full, spec.pos_offset, spec.R, spec.temperature, spec.tau_kl, spec.tau_conf)
+    t3 = time.perf_counter()
+    per_seq = ((t1 - t0) * spec.Hq / len(heads) + (t2 - t1) * spec.R / len(rows) + (t3 - t2))
+    return per_seq * spec.B
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(x, spec, budget_s=12.0):
+    """Full oracle steps of sequence 0 until ~budget_s of host time."""
+    per, n, t0 = [], 0, time.perf_counter()
+    while n == 0 or (time.perf_counter() - t0) < budget_s:
+        per.append(oracle_step(x, spec, b=n % spec.B))
+        n += 1
+        if n >= 20:
+            break
+    sec = float(np.mean(per))
+    return {"value": 1.0 / sec, "unit": "steps/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{n} full fp64 oracle step(s) of one sequence of {spec.name} "
+                      f"(all {spec.Hq} heads, all {spec.R} rows), scaled to the batch of {spec.B}"}
+
+
+# ----------------------------------------------------------------------------- arms
+def run_reference(args, world, rank):
+    """The oracle as the reference arm: bounded samples of the same workload per step."""
+    if rank != 0:
+        return
+    spec = spec_by_name(args.workload)
+    x = W.make_inputs(spec, "cpu", seed=shard_seed(spec, 0))
+    # Per-step sample sized so the whole run takes ~90 s of host time: every
+    # hs-th head and every rs-th verified row of one sequence, select/decide whole.
+    t0 = time.perf_counter()
+    oracle_step(x, spec, 0, spec.Hq, spec.R)  # one head, one row: calibration
+    t_min = max(time.perf_counter() - t0, 1e-3)
+    full = oracle_step(x, spec, 0, 1, 1) / spec.B
+    budget = 90.0 / max(1, args.steps + args.warmup)
+    frac = min(1.0, max(budget - t_min, 0.0) / max(full, 1e-9))
+    hs = max(1, int(round(1.0 / max(frac, 1.0 / spec.Hq))))
+    rs = max(1, int(round(1.0 / max(frac, 1.0 / spec.R))))
+    for _ in range(args.warmup):
+        oracle_step(x, spec, 0, hs, rs)
+    times = [oracle_step(x, spec, k % spec.B, hs, rs) for k in range(args.steps)]
+    sec = float(np.mean(times))
+    value = 1.0 / sec
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "positions_per_s": value * spec.B * spec.R,
+        "config": {"workload": spec.name, "B": spec.B, "L": spec.L, "Hq": spec.Hq,
+                   "Hkv": spec.Hkv, "d": spec.d, "V": spec.V, "R": spec.R, "seeds": spec.k,
+                   "temperature": spec.temperature, "policy": spec.policy},
+        "cpu_baseline": {"value": value, "unit": "steps/s", "cores": blas_threads(),
+                         "kind": "oracle",
+                         "sample": f"per step: heads 0::{hs} of {spec.Hq}, rows 0::{rs} of "
+                                   f"{spec.R} of one sequence, whole select/decide; time "
+                                   f"extrapolated to the full batch of {spec.B}"},
+        "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, world, rank, local):
+    from speculative_verification_cover_b200 import dd
+    from speculative_verification_cover_b200.step import INPUT_KEYS, KERNELS_PER_STEP, VerifyStep
+    dd.lib()  # fail loudly if the library is missing
+    spec = spec_by_name(args.workload)
+    dev = torch.device("cuda", local)
+    x = W.make_inputs(spec, dev, seed=shard_seed(spec, rank))
+    step = VerifyStep(spec, x)
+    step.choose_initial_seeds()
+    step.capture()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        step.replay()
+    torch.cuda.synchronize()
+    assert dd.dd_get_device_error() == dd.DD_OK
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    with ClockSampler(dev.index) as clocks:
+        barrier(world)
+        torch.cuda.synchronize()
+        for k in range(K):
+            flush.zero_()  # L2 flush, outside the per-step event window
+            step.replay(ev[k])
+        torch.cuda.synchronize()
+        barrier(world)
+    step_ms = [e[0].elapsed_time(e[3]) for e in ev]
+    attn_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    ver_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    sel_ms = [e[2].elapsed_time(e[3]) for e in ev]
+    mean = lambda v: float(np.mean(v))
+    ms, a_ms, v_ms, s_ms = max_over_ranks([mean(step_ms), mean(attn_ms), mean(ver_ms),
+                                           mean(sel_ms)], world)
+    assert dd.dd_get_device_error() == dd.DD_OK
+
+    # ---- end to end through the public API: pinned host inputs -> device -> host decisions
+    host = {k: x[k].detach().cpu().pin_memory() for k in INPUT_KEYS}
+    outs = step.result_tensors()
+    host_out = [t.detach().cpu().pin_memory() for t in outs]
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+    Ke = max(3, min(K, 50))
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(Ke)]
+    for k in range(Ke + 2):
+        e = e2e_ev[k - 2] if k >= 2 else None
+        if e:
+            e[0].record()
+        for key in INPUT_KEYS:
+            step.x[key].copy_(host[key], non_blocking=True)
+        step.replay()
+        for t, h in zip(outs, host_out):
+            h.copy_(t, non_blocking=True)
+        if e:
+            e[1].record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks([mean([a.elapsed_time(b) for a, b in e2e_ev])], world)[0]
+
+    hbm, bf16, bf16_s, peak_src = peaks()
+    vbytes, aflops, pflops = algorithmic(spec)
+    achieved = vbytes / (v_ms * 1e-3) / 1e9
+    value = world * 1000.0 / ms
+    line = {
+        "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if spec.dtype == "bf16" else "f32",
+        "data": "synthetic (seeded; shapes and distributions of the named model)",
+        "positions_per_s": value * spec.B * spec.R,
+        "config": {"workload": spec.name, "B": spec.B, "L": spec.L, "Hq": spec.Hq,
+                   "Hkv": spec.Hkv, "d": spec.d, "V": spec.V, "R": spec.R, "seeds": spec.k,
+                   "temperature": spec.temperature, "policy": spec.policy,
+                   "per_rank_batch": spec.B,
+                   "parallelism": f"{world} replica(s), independent batches" if world > 1
+                   else "1 GPU",
+                   "l2": "flushed between steps (256 MiB write outside the step's event "
+                         "window); the logits (%.0f MB) also exceed L2" % (vbytes / 1e6)},
+        "phases_ms": {"attention": a_ms, "verify": v_ms, "select_decide": s_ms},
+        "roofline": {"bound": "hbm", "kernel": "verify_logits_kernel", "achieved": achieved,
+                     "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                     "traffic": recorded_traffic("dd_verify.cu", spec.name),
+                     "algorithmic_bytes": vbytes,
+                     "peak_source": f"MEASURED_PEAKS.json hbm_gbs ({peak_src})"},
+        "attention": {"bound": "tensor", "algorithmic_flop": aflops + pflops,
+                      "achieved_tflops": (aflops + pflops) / (a_ms * 1e-3) / 1e12,
+                      "peak_tflops": bf16, "frac": (aflops + pflops) / (a_ms * 1e-3) / 1e12 / bf16,
+                      "peak_source": f"MEASURED_PEAKS.json bf16_tflops ({peak_src})"},
+        "e2e": {"value": world * 1000.0 / e2e_ms, "unit": "steps/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": KERNELS_PER_STEP * K,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(x, spec)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    step.graphs = None  # release graphs before the process group
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

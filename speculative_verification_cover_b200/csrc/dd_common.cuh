@@ -1,0 +1,105 @@
+// Shared device-side pieces of libdd: the device error word, bounded
+// waits, the Philox4x32-10 generator, and small numeric helpers.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/dd.h"
+
+namespace dd {
+
+// ---------------------------------------------------------------------------
+// Device error word: a kernel whose bounded wait runs out records a dd_status
+// here (first writer wins) and returns; dd_get_device_error() reads and clears
+// it from the host. (libdd is built as one translation unit, libdd.cu, so the
+// definition lives here.)
+__device__ unsigned int g_device_error = 0;
+
+__device__ __forceinline__ void record_error(unsigned int code) {
+  atomicCAS(&g_device_error, 0u, code);
+}
+
+// ---------------------------------------------------------------------------
+// mbarrier helpers (shared::cta). Every wait is bounded by `limit`
+// iterations; on expiry it records DD_ERR_TIMEOUT and returns false.
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t phase) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(phase)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t phase, uint32_t limit) {
+  for (uint32_t it = 0; it < limit; ++it) {
+    if (mbar_try_wait(bar, phase)) return true;
+  }
+  record_error(DD_ERR_TIMEOUT);
+  return false;
+}
+
+// ---------------------------------------------------------------------------
+// Philox4x32-10 (Salmon, Moraes, Dror, Shaw, SC'11): ten rounds of
+//   (x0,x1,x2,x3) -> (hi(M1*x2)^x1^k0, lo(M1*x2), hi(M0*x0)^x3^k1, lo(M0*x0))
+// with the key bumped by the Weyl increments after each round.
+struct PhiloxOut { uint32_t w[4]; };
+
+__device__ __forceinline__ PhiloxOut philox4x32_10(uint32_t c0, uint32_t c1, uint32_t c2,
+                                                   uint32_t c3, uint32_t k0, uint32_t k1) {
+  const uint32_t M0 = 0xD2511F53u, M1 = 0xCD9E8D57u;
+  const uint32_t W0 = 0x9E3779B9u, W1 = 0xBB67AE85u;
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    const uint32_t lo0 = M0 * c0, hi0 = __umulhi(M0, c0);
+    const uint32_t lo1 = M1 * c2, hi1 = __umulhi(M1, c2);
+    const uint32_t n0 = hi1 ^ c1 ^ k0, n2 = hi0 ^ c3 ^ k1;
+    c0 = n0; c1 = lo1; c2 = n2; c3 = lo0;
+    k0 += W0; k1 += W1;
+  }
+  PhiloxOut o;
+  o.w[0] = c0; o.w[1] = c1; o.w[2] = c2; o.w[3] = c3;
+  return o;
+}
+
+// U = (2*(w >> 9) + 1) * 2^-24, exact in fp32, in (0, 1).
+__device__ __forceinline__ float uniform_from_word(uint32_t w) {
+  return __uint2float_rn(2u * (w >> 9) + 1u) * 5.9604644775390625e-08f;
+}
+
+// g = -ln(-ln U). The inner log must be accurate in *relative* terms near
+// U = 1 (where -ln U is tiny and the Gumbel value is large), so it uses the
+// full-precision logf; the outer one only needs absolute accuracy.
+__device__ __forceinline__ float gumbel_from_word(uint32_t w) {
+  const float u = uniform_from_word(w);
+  const float e = -logf(u);
+  return -__logf(e);
+}
+
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+}  // namespace dd

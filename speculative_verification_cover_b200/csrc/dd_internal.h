@@ -1,0 +1,74 @@
+// Internal launcher interface between the C ABI (dd_api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/dd.h"
+
+namespace dd {
+
+struct DeviceInfo {
+  int device;
+  int sm_count;
+  int cc_major, cc_minor;
+  size_t smem_optin;
+};
+// Properties of the current device, cached per device.
+const DeviceInfo& device_info();
+
+// Bound of every device-side wait (iterations).
+uint32_t spin_limit();
+
+struct AttnArgs {
+  const void *q, *k_cur, *v_cur, *k_prev, *v_prev;
+  const uint8_t *is_seed, *is_masked, *is_new;
+  int B, L, Hq, Hkv, d;
+  float scale;          // softmax scale (natural units)
+  dd_dtype dtype;
+  int accumulate;
+  void* out;
+  float* lse;
+  float *d_in, *d_out;
+  // workspace carve-up
+  float* dout_part;     // [B, Hq, L]
+  float* din_part;      // [B, Hq, L]
+  int32_t* mrows;       // [B, L] masked rows of each sequence, ascending
+  int32_t* mcount;      // [B]
+};
+
+// Workspace layout shared by the entry point and the kernels.
+struct AttnWorkspace {
+  size_t dout_off, din_off, mrows_off, mcount_off, total;
+};
+AttnWorkspace attn_workspace_layout(int B, int L, int Hq);
+
+cudaError_t launch_attention(const AttnArgs& a, cudaStream_t stream);
+
+cudaError_t launch_verify_logits(const void* lt, const void* lm, dd_dtype dtype, int B, int R,
+                                 int V, int64_t ld, int pos_offset, float temperature,
+                                 uint64_t seed, uint64_t step, const dd_row_stats& out,
+                                 cudaStream_t stream);
+
+cudaError_t launch_coupled_gumbel(uint64_t seed, uint64_t step, int B, int R, int V, int64_t ld,
+                                  int pos_offset, float* g, cudaStream_t stream);
+
+cudaError_t launch_select_seeds(const float* entropy, int R, int pos_offset, const float* d_in,
+                                const float* d_out, const uint8_t* eligible, int B, int L, int k,
+                                int32_t* seeds, uint8_t* is_seed, float* score,
+                                cudaStream_t stream);
+
+cudaError_t launch_decide(const dd_decide_params& p, const int32_t* tokens,
+                          const uint8_t* is_seed, const uint8_t* eligible,
+                          const dd_row_stats& stats, int B, int L, int R, int pos_offset,
+                          uint8_t* decision, int32_t* new_tokens, uint8_t* accepted,
+                          cudaStream_t stream);
+
+cudaError_t launch_selftest_wait(uint32_t limit, cudaStream_t stream);
+
+// Largest L dd_select_seeds handles (keys of one sequence live in shared memory).
+constexpr int kSelectMaxL = 24576;
+constexpr int kSelectMaxK = 1024;
+
+}  // namespace dd

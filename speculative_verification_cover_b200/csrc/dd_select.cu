@@ -1,0 +1,222 @@
+// Stability-aware seed selection (dd_select_seeds), the verification
+// decisions (dd_decide) and the bounded-wait self-test.
+#include "dd_common.cuh"
+#include "dd_internal.h"
+
+namespace dd {
+
+namespace {
+
+constexpr int kSelThreads = 1024;
+
+// Order-preserving map of a float onto uint32 (larger float -> larger key).
+__device__ __forceinline__ uint32_t orderable(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// One CTA per sequence.
+//   score_i = u_i (1 + d_in_i) / (1 + d_out_i) on eligible positions with a row.
+// Candidates get the 64-bit key (orderable(score) << 32) | (0xFFFFFFFF - i):
+// keys are distinct, larger key = higher score, then lower position. The k-th
+// largest key is found by an MSB-first radix select (8 passes of 8 bits) over
+// keys in shared memory; the chosen positions are ranked by counting.
+__global__ void __launch_bounds__(kSelThreads)
+select_seeds_kernel(const float* __restrict__ entropy, int R, int pos_offset,
+                    const float* __restrict__ d_in, const float* __restrict__ d_out,
+                    const uint8_t* __restrict__ eligible, int L, int k,
+                    int32_t* __restrict__ seeds, uint8_t* __restrict__ is_seed,
+                    float* __restrict__ score) {
+  extern __shared__ unsigned long long keys[];  // [L]; 0 = not a candidate
+  __shared__ unsigned int hist[256];
+  __shared__ unsigned int warp_tot[kSelThreads / 32];
+  __shared__ unsigned long long prefix_s;
+  __shared__ int need_s, ncand_s, nsel_s;
+  __shared__ unsigned long long chosen[kSelectMaxK];
+
+  const int b = blockIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) { ncand_s = 0; nsel_s = 0; }
+  __syncthreads();
+  int my_cand = 0;
+  for (int i = threadIdx.x; i < L; i += blockDim.x) {
+    const int64_t bi = (int64_t)b * L + i;
+    const int r = i - pos_offset;
+    float s = -INFINITY;
+    unsigned long long key = 0ull;
+    if (eligible[bi] && r >= 0 && r < R) {
+      const float u = entropy[(int64_t)b * R + r];
+      s = u * (1.f + d_in[bi]) / (1.f + d_out[bi]);
+      key = ((unsigned long long)orderable(s) << 32) | (0xFFFFFFFFu - (uint32_t)i);
+      ++my_cand;
+    }
+    keys[i] = key;
+    if (score) score[bi] = s;
+  }
+  atomicAdd(&ncand_s, my_cand);
+  __syncthreads();
+  const int ncand = ncand_s;
+  const int kk = k < ncand ? k : ncand;
+  unsigned long long thresh = 1ull;  // select keys >= thresh (all candidates by default)
+  if (kk > 0 && kk < ncand) {
+    unsigned long long prefix = 0ull;
+    int need = kk;  // how many keys >= the final threshold remain to be found below prefix
+    for (int shift = 56; shift >= 0; shift -= 8) {
+      for (int t = threadIdx.x; t < 256; t += blockDim.x) hist[t] = 0u;
+      __syncthreads();
+      const unsigned long long hmask = shift == 56 ? 0ull : (~0ull << (shift + 8));
+      for (int i = threadIdx.x; i < L; i += blockDim.x) {
+        const unsigned long long key = keys[i];
+        if (key != 0ull && (key & hmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+      }
+      __syncthreads();
+      // thread t < 256 takes digit 255 - t; inclusive scan gives #keys with digit >= 255 - t
+      unsigned int c = 0u, incl = 0u;
+      if (threadIdx.x < 256) {
+        c = hist[255 - threadIdx.x];
+        incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const unsigned int t2 = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += t2;
+        }
+        if (lane == 31) warp_tot[warp] = incl;
+      }
+      __syncthreads();
+      if (threadIdx.x < 256) {
+        for (int w = 0; w < warp; ++w) incl += warp_tot[w];
+        if (incl >= (unsigned)need && incl - c < (unsigned)need) {
+          const unsigned long long digit = 255 - threadIdx.x;
+          prefix_s = prefix | (digit << shift);
+          need_s = need - (int)(incl - c);
+        }
+      }
+      __syncthreads();
+      prefix = prefix_s;
+      need = need_s;
+      __syncthreads();
+    }
+    thresh = prefix;  // the kk-th largest key itself
+  }
+  // collect the chosen keys
+  for (int i = threadIdx.x; i < L; i += blockDim.x) {
+    const unsigned long long key = keys[i];
+    const bool sel = kk > 0 && key != 0ull && key >= thresh;
+    if (sel) chosen[atomicAdd(&nsel_s, 1)] = key;
+    if (is_seed) is_seed[(int64_t)b * L + i] = sel ? 1 : 0;
+  }
+  __syncthreads();
+  const int nsel = nsel_s;
+  for (int t = threadIdx.x; t < nsel; t += blockDim.x) {
+    const unsigned long long key = chosen[t];
+    int rank = 0;
+    for (int u = 0; u < nsel; ++u) rank += chosen[u] > key;
+    seeds[(int64_t)b * k + rank] = (int32_t)(0xFFFFFFFFu - (uint32_t)(key & 0xFFFFFFFFull));
+  }
+  for (int t = nsel + threadIdx.x; t < k; t += blockDim.x) seeds[(int64_t)b * k + t] = -1;
+}
+
+// One CTA per sequence; accepted[b] = all decided positions KEEP.
+__global__ void __launch_bounds__(256)
+decide_kernel(dd_decide_params p, const int32_t* __restrict__ tokens,
+              const uint8_t* __restrict__ is_seed, const uint8_t* __restrict__ eligible,
+              dd_row_stats st, int L, int R, int pos_offset, uint8_t* __restrict__ decision,
+              int32_t* __restrict__ new_tokens, uint8_t* __restrict__ accepted) {
+  const int b = blockIdx.x;
+  const bool sampled = p.temperature > 0.f;
+  int all_keep = 1;
+  for (int i = threadIdx.x; i < L; i += blockDim.x) {
+    const int64_t bi = (int64_t)b * L + i;
+    const int r = i - pos_offset;
+    const int32_t cur = tokens[bi];
+    const uint8_t* domain = p.policy == DD_POLICY_COVER ? is_seed : eligible;
+    const bool in = r >= 0 && r < R && domain != nullptr && domain[bi];
+    uint8_t dcs = DD_NONE;
+    int32_t tok = cur;
+    if (in) {
+      const int64_t row = (int64_t)b * R + r;
+      const int32_t pred = sampled ? st.sample_t[row] : st.argmax_t[row];
+      switch (p.policy) {
+        case DD_POLICY_TRUST:
+          dcs = DD_KEEP;
+          break;
+        case DD_POLICY_KL:
+          dcs = st.kl_dt[row] > p.tau_kl ? DD_REMASK : DD_KEEP;
+          break;
+        case DD_POLICY_CONF:
+          dcs = st.conf_t[row] < p.tau_conf ? DD_REMASK : DD_KEEP;
+          break;
+        case DD_POLICY_COVER:
+          if (pred == cur) dcs = DD_KEEP;
+          else dcs = st.p_sample_t[row] >= p.tau_conf ? DD_REPLACE : DD_REMASK;
+          break;
+        case DD_POLICY_COUPLED: {
+          const int32_t sd = sampled ? st.sample_d[row] : st.argmax_d[row];
+          if (sd == pred) dcs = DD_KEEP;
+          else if (p.tau_kl > 0.f && st.kl_dt[row] > p.tau_kl) dcs = DD_REMASK;
+          else dcs = DD_REPLACE;
+          break;
+        }
+        default:
+          break;
+      }
+      if (dcs == DD_REPLACE || (dcs == DD_KEEP && p.policy == DD_POLICY_COUPLED)) tok = pred;
+      else if (dcs == DD_REMASK) tok = DD_MASK_TOKEN;
+      if (dcs != DD_KEEP) all_keep = 0;
+    }
+    decision[bi] = dcs;
+    new_tokens[bi] = tok;
+  }
+  const int acc = __syncthreads_and(all_keep);
+  if (accepted && threadIdx.x == 0) accepted[b] = (uint8_t)acc;
+}
+
+// Failure-detection self-test: wait on an mbarrier that nobody arrives on.
+__global__ void selftest_wait_kernel(uint32_t limit) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait_bounded(&bar, 0, limit);
+  __syncthreads();
+}
+
+}  // namespace
+
+cudaError_t launch_select_seeds(const float* entropy, int R, int pos_offset, const float* d_in,
+                                const float* d_out, const uint8_t* eligible, int B, int L, int k,
+                                int32_t* seeds, uint8_t* is_seed, float* score,
+                                cudaStream_t stream) {
+  const size_t smem = (size_t)L * sizeof(unsigned long long);
+  static thread_local int configured_for = -1;
+  const DeviceInfo& dev = device_info();
+  if (configured_for != dev.device) {
+    cudaError_t e = cudaFuncSetAttribute(select_seeds_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)(kSelectMaxL * sizeof(unsigned long long)));
+    if (e != cudaSuccess) return e;
+    configured_for = dev.device;
+  }
+  select_seeds_kernel<<<B, kSelThreads, smem, stream>>>(entropy, R, pos_offset, d_in, d_out,
+                                                        eligible, L, k, seeds, is_seed, score);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decide(const dd_decide_params& p, const int32_t* tokens,
+                          const uint8_t* is_seed, const uint8_t* eligible,
+                          const dd_row_stats& stats, int B, int L, int R, int pos_offset,
+                          uint8_t* decision, int32_t* new_tokens, uint8_t* accepted,
+                          cudaStream_t stream) {
+  decide_kernel<<<B, 256, 0, stream>>>(p, tokens, is_seed, eligible, stats, L, R, pos_offset,
+                                       decision, new_tokens, accepted);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_selftest_wait(uint32_t limit, cudaStream_t stream) {
+  selftest_wait_kernel<<<1, 32, 0, stream>>>(limit);
+  return cudaGetLastError();
+}
+
+}  // namespace dd

@@ -1,0 +1,239 @@
+"""ctypes binding of libdd.so (include/dd.h), one Python function per C entry point.
+
+Argument marshalling only: sizes are read off the tensors, pointers passed
+as `data_ptr()`, the stream defaults to torch's current CUDA stream. Every
+computation runs in libdd's CUDA kernels; there is no CPU fallback -- CPU
+tensors, a missing library or a non-OK status raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass, fields
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdd.so")
+
+DD_OK, DD_ERR_INVALID_ARG, DD_ERR_UNSUPPORTED, DD_ERR_CUDA, DD_ERR_TIMEOUT = range(5)
+DD_F32, DD_BF16 = 0, 1
+POLICIES = {"trust": 0, "kl": 1, "conf": 2, "cover": 3, "coupled": 4}
+DD_NONE, DD_KEEP, DD_REPLACE, DD_REMASK = 0, 1, 2, 3
+DD_MASK_TOKEN = -1
+
+# Every symbol include/dd.h declares.
+EXPORTED = (
+    "dd_dualview_attention", "dd_dualview_attention_workspace_size", "dd_verify_logits",
+    "dd_coupled_gumbel", "dd_select_seeds", "dd_decide", "dd_status_string",
+    "dd_get_device_error", "dd_set_spin_limit", "dd_selftest_bounded_wait",
+)
+
+
+class DDError(RuntimeError):
+    def __init__(self, fn, status):
+        self.status = status
+        super().__init__(f"{fn} failed: {status_string(status)} ({status})")
+
+
+class _RowStats(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "lse_t", "lse_d", "conf_t", "p_sample_t", "entropy_t", "kl_dt",
+        "argmax_t", "argmax_d", "sample_t", "sample_d")]
+
+
+class _DecideParams(ctypes.Structure):
+    _fields_ = [("policy", ctypes.c_int), ("tau_kl", ctypes.c_float),
+                ("tau_conf", ctypes.c_float), ("temperature", ctypes.c_float)]
+
+
+_lib = None
+
+
+def lib():
+    """Load libdd.so (once). Raises ImportError if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m speculative_verification_cover_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I, I64, U64, F, SZ = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_uint64,
+                             ctypes.c_float, ctypes.c_size_t)
+    L.dd_dualview_attention.argtypes = [P] * 8 + [I] * 5 + [F, I, I] + [P] * 5 + [SZ, P]
+    L.dd_dualview_attention.restype = I
+    L.dd_dualview_attention_workspace_size.argtypes = [I] * 5
+    L.dd_dualview_attention_workspace_size.restype = SZ
+    L.dd_verify_logits.argtypes = [P, P, I, I, I, I, I64, I, F, U64, U64,
+                                   ctypes.POINTER(_RowStats), P]
+    L.dd_verify_logits.restype = I
+    L.dd_coupled_gumbel.argtypes = [U64, U64, I, I, I, I64, I, P, P]
+    L.dd_coupled_gumbel.restype = I
+    L.dd_select_seeds.argtypes = [P, I, I, P, P, P, I, I, I, P, P, P, P]
+    L.dd_select_seeds.restype = I
+    L.dd_decide.argtypes = [ctypes.POINTER(_DecideParams), P, P, P, ctypes.POINTER(_RowStats),
+                            I, I, I, I, P, P, P, P]
+    L.dd_decide.restype = I
+    L.dd_status_string.argtypes = [I]
+    L.dd_status_string.restype = ctypes.c_char_p
+    L.dd_get_device_error.argtypes = [P]
+    L.dd_get_device_error.restype = I
+    L.dd_set_spin_limit.argtypes = [ctypes.c_uint32]
+    L.dd_set_spin_limit.restype = ctypes.c_uint32
+    L.dd_selftest_bounded_wait.argtypes = [ctypes.c_uint32, P]
+    L.dd_selftest_bounded_wait.restype = I
+    _lib = L
+    return L
+
+
+def status_string(status: int) -> str:
+    return lib().dd_status_string(int(status)).decode()
+
+
+def _check(fn, status):
+    if status != DD_OK:
+        raise DDError(fn, status)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("expected a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError("libdd takes device memory: tensor is on the CPU")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _dtype_code(t):
+    if t.dtype == torch.float32:
+        return DD_F32
+    if t.dtype == torch.bfloat16:
+        return DD_BF16
+    raise ValueError(f"unsupported dtype {t.dtype}")
+
+
+@dataclass
+class RowStats:
+    """Per-row outputs of dd_verify_logits, each a [B, R] device tensor (or None)."""
+    lse_t: torch.Tensor | None = None
+    lse_d: torch.Tensor | None = None
+    conf_t: torch.Tensor | None = None
+    p_sample_t: torch.Tensor | None = None
+    entropy_t: torch.Tensor | None = None
+    kl_dt: torch.Tensor | None = None
+    argmax_t: torch.Tensor | None = None
+    argmax_d: torch.Tensor | None = None
+    sample_t: torch.Tensor | None = None
+    sample_d: torch.Tensor | None = None
+
+    @classmethod
+    def empty(cls, B, R, device="cuda"):
+        f = dict(dtype=torch.float32, device=device)
+        i = dict(dtype=torch.int32, device=device)
+        return cls(*(torch.empty(B, R, **f) for _ in range(6)),
+                   *(torch.empty(B, R, **i) for _ in range(4)))
+
+    def _c(self):
+        return _RowStats(*(_ptr(getattr(self, f.name)) for f in fields(self)))
+
+
+def dd_dualview_attention_workspace_size(B, L, Hq, Hkv, d) -> int:
+    return int(lib().dd_dualview_attention_workspace_size(B, L, Hq, Hkv, d))
+
+
+def dd_dualview_attention(q, k_cur, v_cur, k_prev, v_prev, is_seed, is_masked, is_new,
+                          out, lse, d_in=None, d_out=None, workspace=None, softmax_scale=0.0,
+                          accumulate_stats=False, stream=None):
+    """q [B,L,Hq,d]; k/v [B,L,Hkv,d]; masks [B,L] uint8; out like q; lse [B,Hq,L] fp32;
+    d_in, d_out [B,L] fp32; workspace: uint8 device tensor of
+    dd_dualview_attention_workspace_size(...) bytes."""
+    B, L, Hq, d = q.shape
+    Hkv = k_cur.shape[2]
+    nbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = lib().dd_dualview_attention(
+        _ptr(q), _ptr(k_cur), _ptr(v_cur), _ptr(k_prev), _ptr(v_prev), _ptr(is_seed),
+        _ptr(is_masked), _ptr(is_new), B, L, Hq, Hkv, d, float(softmax_scale), _dtype_code(q),
+        int(bool(accumulate_stats)), _ptr(out), _ptr(lse), _ptr(d_in), _ptr(d_out),
+        _ptr(workspace), nbytes, _stream(stream))
+    _check("dd_dualview_attention", st)
+
+
+def dd_verify_logits(logits_t, logits_d, out: RowStats, pos_offset=0, temperature=0.0, seed=0,
+                     step=0, stream=None):
+    """logits [B,R,V]; a view narrowed from a wider [B,R,ld] buffer is accepted
+    (the row stride ld is read from the tensor). out: RowStats of [B,R] tensors."""
+    B, R, V = logits_t.shape
+    if logits_t.stride(2) != 1 or logits_t.stride(0) != R * logits_t.stride(1):
+        raise ValueError("logits must be [B,R,V] with unit vocabulary stride and packed rows")
+    if logits_d.shape != logits_t.shape or logits_d.stride() != logits_t.stride():
+        raise ValueError("verifier and drafter logits must have the same shape and strides")
+    if not (logits_t.is_cuda and logits_d.is_cuda):
+        raise ValueError("libdd takes device memory: logits are on the CPU")
+    ld = logits_t.stride(1)
+    st = lib().dd_verify_logits(
+        ctypes.c_void_p(logits_t.data_ptr()), ctypes.c_void_p(logits_d.data_ptr()),
+        _dtype_code(logits_t), B, R, V, ld, int(pos_offset), float(temperature),
+        int(seed) & (2**64 - 1), int(step) & (2**64 - 1), ctypes.byref(out._c()),
+        _stream(stream))
+    _check("dd_verify_logits", st)
+
+
+def dd_coupled_gumbel(g, seed=0, step=0, pos_offset=0, stream=None):
+    """Fill g [B,R,V] fp32 with the shared Gumbel noise of dd_verify_logits."""
+    B, R, V = g.shape
+    st = lib().dd_coupled_gumbel(int(seed) & (2**64 - 1), int(step) & (2**64 - 1), B, R, V,
+                                 g.stride(1), int(pos_offset), _ptr(g), _stream(stream))
+    _check("dd_coupled_gumbel", st)
+
+
+def dd_select_seeds(entropy, pos_offset, d_in, d_out, eligible, seeds, is_seed=None, score=None,
+                    stream=None):
+    """entropy [B,R]; d_in, d_out [B,L] fp32; eligible [B,L] u8; seeds [B,k] int32 out."""
+    B, L = d_in.shape
+    R = entropy.shape[1] if entropy is not None else 0
+    k = seeds.shape[1] if seeds is not None else 0
+    st = lib().dd_select_seeds(_ptr(entropy), R, int(pos_offset), _ptr(d_in), _ptr(d_out),
+                               _ptr(eligible), B, L, k, _ptr(seeds), _ptr(is_seed), _ptr(score),
+                               _stream(stream))
+    _check("dd_select_seeds", st)
+
+
+def dd_decide(policy, tokens, is_seed, eligible, stats: RowStats, pos_offset, decision,
+              new_tokens, accepted=None, tau_kl=0.5, tau_conf=0.9, temperature=0.0, stream=None):
+    """tokens [B,L] int32; stats from dd_verify_logits ([B,R]); decision [B,L] u8,
+    new_tokens [B,L] int32, accepted [B] u8 outputs."""
+    B, L = tokens.shape
+    ref = stats.argmax_t if stats.argmax_t is not None else stats.sample_t
+    R = ref.shape[1]
+    p = _DecideParams(POLICIES[policy] if isinstance(policy, str) else int(policy),
+                      float(tau_kl), float(tau_conf), float(temperature))
+    st = lib().dd_decide(ctypes.byref(p), _ptr(tokens), _ptr(is_seed), _ptr(eligible),
+                         ctypes.byref(stats._c()), B, L, R, int(pos_offset), _ptr(decision),
+                         _ptr(new_tokens), _ptr(accepted), _stream(stream))
+    _check("dd_decide", st)
+
+
+def dd_get_device_error(stream=None) -> int:
+    """Synchronise the stream; return and clear the device error word."""
+    return int(lib().dd_get_device_error(_stream(stream)))
+
+
+def dd_set_spin_limit(limit: int) -> int:
+    return int(lib().dd_set_spin_limit(int(limit)))
+
+
+def dd_selftest_bounded_wait(spin_limit: int, stream=None):
+    _check("dd_selftest_bounded_wait", lib().dd_selftest_bounded_wait(int(spin_limit),
+                                                                      _stream(stream)))

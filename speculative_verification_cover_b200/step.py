@@ -1,0 +1,124 @@
+"""One verification step over device-resident buffers, built on the C ABI.
+
+A step is the four library calls in order, on one stream:
+  1. dd_dualview_attention  -- dual-view attention (one layer) with d_in, d_out
+  2. dd_verify_logits       -- per-row statistics and coupled samples
+  3. dd_select_seeds        -- the next step's seed set from u, d_in, d_out
+  4. dd_decide              -- KEEP / REPLACE / REMASK
+Buffers are allocated once (torch, caller side); the library itself never
+allocates. The three phases can be captured into CUDA graphs and replayed.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import dd
+from .workloads import WorkloadSpec
+
+INPUT_KEYS = ("q", "k_cur", "v_cur", "k_prev", "v_prev", "is_seed", "is_masked", "is_new",
+              "eligible", "tokens", "logits_t", "logits_d")
+# Our kernels per step: masked-row compaction, attention pass 1, pass 2, two
+# head reductions, verify, select, decide.
+KERNELS_PER_STEP = 8
+
+
+class VerifyStep:
+    def __init__(self, spec: WorkloadSpec, inputs: dict, seed: int = 2024, step_index: int = 1,
+                 use_seeds: bool = True):
+        self.spec = spec
+        self.x = {k: inputs[k] for k in INPUT_KEYS}
+        dev = self.x["q"].device
+        B, L, Hq, Hkv, d, R = spec.B, spec.L, spec.Hq, spec.Hkv, spec.d, spec.R
+        self.seed, self.step_index = seed, step_index
+        self.use_seeds = use_seeds and spec.k > 0
+        self.out = torch.empty_like(self.x["q"])
+        self.lse = torch.empty(B, Hq, L, device=dev)
+        self.d_in = torch.empty(B, L, device=dev)
+        self.d_out = torch.empty(B, L, device=dev)
+        self.ws = torch.empty(dd.dd_dualview_attention_workspace_size(B, L, Hq, Hkv, d),
+                              dtype=torch.uint8, device=dev)
+        self.stats = dd.RowStats.empty(B, R, dev)
+        self.k = max(spec.k, 1)
+        self.next_seeds = torch.empty(B, self.k, dtype=torch.int32, device=dev)
+        self.next_is_seed = torch.empty(B, L, dtype=torch.uint8, device=dev)
+        self.score = torch.empty(B, L, device=dev)
+        self.decision = torch.empty(B, L, dtype=torch.uint8, device=dev)
+        self.new_tokens = torch.empty(B, L, dtype=torch.int32, device=dev)
+        self.accepted = torch.empty(B, dtype=torch.uint8, device=dev)
+        self.graphs = None
+
+    # --- the four calls
+    def attention(self):
+        x = self.x
+        dd.dd_dualview_attention(
+            x["q"], x["k_cur"], x["v_cur"], x["k_prev"] if self.use_seeds else None,
+            x["v_prev"] if self.use_seeds else None, x["is_seed"] if self.use_seeds else None,
+            x["is_masked"], x["is_new"], self.out, self.lse, self.d_in, self.d_out, self.ws)
+
+    def verify(self):
+        s = self.spec
+        dd.dd_verify_logits(self.x["logits_t"], self.x["logits_d"], self.stats,
+                            pos_offset=s.pos_offset, temperature=s.temperature, seed=self.seed,
+                            step=self.step_index)
+
+    def select_and_decide(self):
+        s, x = self.spec, self.x
+        dd.dd_select_seeds(self.stats.entropy_t, s.pos_offset, self.d_in, self.d_out,
+                           x["eligible"], self.next_seeds, self.next_is_seed, self.score)
+        dd.dd_decide(s.policy, x["tokens"], x["is_seed"], x["eligible"], self.stats,
+                     s.pos_offset, self.decision, self.new_tokens, self.accepted,
+                     tau_kl=s.tau_kl, tau_conf=s.tau_conf, temperature=s.temperature)
+
+    def __call__(self):
+        self.attention()
+        self.verify()
+        self.select_and_decide()
+
+    def choose_initial_seeds(self):
+        """Pass 0 with an empty seed set, then the stability score picks the seeds the
+        step will verify (the seeds of step t come from the scores of step t-1)."""
+        if self.spec.k == 0:
+            return
+        keep = self.use_seeds
+        self.use_seeds = False
+        self.attention()
+        self.verify()
+        s = self.spec
+        dd.dd_select_seeds(self.stats.entropy_t, s.pos_offset, self.d_in, self.d_out,
+                           self.x["eligible"], self.next_seeds, self.next_is_seed, self.score)
+        self.x["is_seed"].copy_(self.next_is_seed)
+        self.use_seeds = keep
+
+    # --- CUDA graphs
+    def capture(self):
+        self()  # warm every kernel (lazy attribute set-up happens outside capture)
+        torch.cuda.synchronize()
+        graphs = []
+        for fn in (self.attention, self.verify, self.select_and_decide):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                fn()
+            graphs.append(g)
+        torch.cuda.synchronize()
+        self.graphs = graphs
+        return graphs
+
+    def replay(self, events=None):
+        """Replay the captured phases; events (4 timing events or None) are recorded
+        before attention, before verify, after verify and at the end."""
+        ga, gv, gs = self.graphs
+        if events:
+            events[0].record()
+        ga.replay()
+        if events:
+            events[1].record()
+        gv.replay()
+        if events:
+            events[2].record()
+        gs.replay()
+        if events:
+            events[3].record()
+
+    def result_tensors(self):
+        """What a caller reads back after a step."""
+        return (self.decision, self.new_tokens, self.accepted, self.next_seeds)

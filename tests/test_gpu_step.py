@@ -1,0 +1,64 @@
+"""One whole verification step through the C ABI against the oracle (GPU):
+dual-view attention -> vocabulary verification -> seed selection -> decisions."""
+import numpy as np
+import pytest
+import torch
+
+from speculative_verification_cover_b200 import dd
+from speculative_verification_cover_b200 import workloads as W
+from tests import parity as PA
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("T,policy", [(0.0, "cover"), (1.0, "cover"), (0.0, "kl"),
+                                      (0.0, "conf"), (1.0, "coupled"), (0.0, "trust")])
+def test_tiny_step(T, policy):
+    spec = W.TINY_F32.replace(temperature=T, policy=policy)
+    x = W.make_inputs(spec, "cpu")
+    xg = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+    B, L, Hq, Hkv, d, R, off = spec.B, spec.L, spec.Hq, spec.Hkv, spec.d, spec.R, spec.pos_offset
+    out = torch.empty_like(xg["q"])
+    lse = torch.empty(B, Hq, L, device="cuda")
+    d_in = torch.empty(B, L, device="cuda")
+    d_out = torch.empty(B, L, device="cuda")
+    ws = torch.empty(dd.dd_dualview_attention_workspace_size(B, L, Hq, Hkv, d),
+                     dtype=torch.uint8, device="cuda")
+    dd.dd_dualview_attention(xg["q"], xg["k_cur"], xg["v_cur"], xg["k_prev"], xg["v_prev"],
+                             xg["is_seed"], xg["is_masked"], xg["is_new"], out, lse, d_in, d_out,
+                             ws)
+    stats = dd.RowStats.empty(B, R)
+    dd.dd_verify_logits(xg["logits_t"], xg["logits_d"], stats, pos_offset=off, temperature=T,
+                        seed=0, step=0)
+    seeds = torch.empty(B, spec.k, dtype=torch.int32, device="cuda")
+    next_seed = torch.empty(B, L, dtype=torch.uint8, device="cuda")
+    dd.dd_select_seeds(stats.entropy_t, off, d_in, d_out, xg["eligible"], seeds, next_seed)
+    dec = torch.empty(B, L, dtype=torch.uint8, device="cuda")
+    newt = torch.empty(B, L, dtype=torch.int32, device="cuda")
+    acc = torch.empty(B, dtype=torch.uint8, device="cuda")
+    dd.dd_decide(policy, xg["tokens"], xg["is_seed"], xg["eligible"], stats, off, dec, newt, acc,
+                 tau_kl=spec.tau_kl, tau_conf=spec.tau_conf, temperature=T)
+    torch.cuda.synchronize()
+    assert dd.dd_get_device_error() == dd.DD_OK
+
+    # oracle, step by step, on the same inputs
+    wo, wl, wdin, wdout = PA.oracle_attention_seq(x, 0)
+    PA.assert_close("out", PA.np64(out[0]), wo, 0, 1e-4)
+    PA.assert_close("d_in", PA.np64(d_in[0]), wdin, PA.MASS_RTOL, PA.MASS_ATOL)
+    PA.assert_close("d_out", PA.np64(d_out[0]), wdout, PA.MASS_RTOL, PA.MASS_ATOL)
+    rows = np.arange(R)
+    ws_ = PA.oracle_verify(x["logits_t"], x["logits_d"], rows, R, off, T, 0, 0)
+    near_rows = PA.compare_verify(stats, ws_, rows, T)
+    u = np.zeros(L)
+    u[off:] = ws_["entropy_t"]
+    want_seeds, want_is, _, margin = PA.oracle_select(u, wdin, wdout, PA.npi(x["eligible"][0]),
+                                                      spec.k)
+    if margin >= 1e-3:  # GPU scores come from GPU statistics: allow their tolerance
+        assert np.array_equal(PA.npi(next_seed[0]), want_is)
+    wd, wt, wa, near = PA.oracle_decide(policy, PA.npi(x["tokens"][0]), PA.npi(x["is_seed"][0]),
+                                        PA.npi(x["eligible"][0]), ws_, off, R, T, spec.tau_kl,
+                                        spec.tau_conf)
+    ok = ~near
+    assert np.array_equal(PA.npi(dec[0])[ok], wd[ok].astype(np.int64))
+    assert np.array_equal(PA.npi(newt[0])[ok], wt[ok].astype(np.int64))
+    assert near_rows + int(near.sum()) <= 2
