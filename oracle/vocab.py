@@ -42,7 +42,10 @@ def _argmax_lowest(x):
 
 
 def _top2_gap(x):
-    """Gap between the largest and the second largest entry of each row."""
+    """Gap between the largest and the second largest entry of each row
+    (infinite when a row has a single entry: there is no runner-up)."""
+    if x.shape[-1] < 2:
+        return np.full(x.shape[:-1], np.inf)
     part = -np.partition(-x, 1, axis=-1)[..., :2]
     return part[..., 0] - part[..., 1]
 

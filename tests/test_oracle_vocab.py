@@ -99,3 +99,11 @@ def test_verify_rows_sampled_probability():
     out = vocab.verify_rows(l, m, 1.0, seed=5, step=1, b=0, positions=np.arange(8) + 3)
     p_t = special.softmax(l, axis=1)
     np.testing.assert_allclose(out["p_sample_t"], p_t[np.arange(8), out["sample_t"]], rtol=1e-12)
+
+
+def test_single_entry_vocabulary():
+    l = np.array([[1.5], [-2.0]])
+    out = vocab.verify_rows(l, l + 1, 1.0, seed=0, step=0, b=0, positions=np.arange(2))
+    assert list(out["sample_t"]) == [0, 0] and np.all(np.isinf(out["margin_t"]))
+    np.testing.assert_allclose(out["entropy_t"], 0, atol=1e-15)
+    np.testing.assert_allclose(out["conf_t"], 1.0)
