@@ -337,6 +337,15 @@ cudaError_t launch_simt(const AttnArgs& a, cudaStream_t stream) {
 
 }  // namespace
 
+cudaError_t launch_simt_pass2_bf16(const AttnArgs& a, cudaStream_t stream) {
+  dim3 g2((a.L + kCols - 1) / kCols, a.Hq, a.B);
+  if (a.d == 64)
+    simt_pass2_kernel<__nv_bfloat16, 64><<<g2, 128, 0, stream>>>(a);
+  else
+    simt_pass2_kernel<__nv_bfloat16, 128><<<g2, 128, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_attention_tc(const AttnArgs& a, cudaStream_t stream, bool* handled);
 
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t stream) {

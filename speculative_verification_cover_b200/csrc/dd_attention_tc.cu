@@ -1,14 +1,509 @@
-// Tensor-core (sm_100a) dual-view attention for bf16 inputs.
-#include "dd_common.cuh"
+// Tensor-core (sm_100a, tcgen05) dual-view attention for bf16 inputs.
+//
+// Pass 1, one CTA per (128 query rows, head, sequence), warp-specialised:
+//   warp 0      producer: TMA loads of the Q tile and of K/V tiles (128 columns,
+//               two stages) from k_cur / v_cur; then, per tile, overwrites the
+//               rows of seed columns with the step t-1 cache (k_prev / v_prev,
+//               plain loads + swizzled shared stores) -- the drafting view; and
+//               writes the tile's "newly written" flags into a small B operand
+//               whose rows are [1, is_new, 0, ...].
+//   warp 1      MMA issuer (one thread): S = Q K^T into a double-buffered TMEM
+//               accumulator; O += P V and [l, l_new] += P [1, is_new]^T, i.e. the
+//               row sum and the mass on newly written columns come out of the
+//               tensor core with the same bf16 P that weights V.
+//   warps 2-5   softmax (one thread per query row = TMEM lane): online max with
+//               a lazy rescale (O is rescaled in TMEM only when the running max
+//               grows by more than 2^8), P = exp2(S*scale*log2e - m) as bf16 into
+//               shared memory. A seed query's own column is masked in the loop and
+//               merged back afterwards from k_cur / v_cur (leave-one-out
+//               diagonal). Epilogue: out = O / l, lse, d_out partial = l_new / l.
+// Every wait is bounded; on expiry the kernel records DD_ERR_TIMEOUT and winds down.
+#include <cudaTypedefs.h>
+
 #include "dd_internal.h"
+#include "dd_tc.cuh"
 
 namespace dd {
 
+namespace {
+
+using namespace tc;
+
+constexpr int kBM = 128;
+constexpr int kBN = 128;
+constexpr int kStages = 2;
+constexpr int kP1Threads = 192;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kAtom = 128 * 128;  // one 128-row x 128-byte swizzle atom column
+
+template <int D>
+struct P1Layout {
+  static constexpr int kTile = (D / 64) * kAtom;  // 128 x D bf16
+  static constexpr int kQ = 0;
+  static constexpr int kK = kQ + kTile;
+  static constexpr int kV = kK + kStages * kTile;
+  static constexpr int kP = kV + kStages * kTile;
+  static constexpr int kB2 = kP + 2 * kAtom;          // P: 128 rows x 128 columns bf16
+  static constexpr int kB2Bytes = 2 * 16 * 128;       // 16 rows x 128 columns bf16
+  static constexpr int kBar = kB2 + kStages * kB2Bytes;
+  static constexpr int kBytes = kBar + 256;
+  // TMEM columns
+  static constexpr uint32_t kS0 = 0, kS1 = 128, kO = 256, kSt = 256 + D;
+};
+
+struct P1Bars {
+  uint64_t q_full;
+  uint64_t kv_full[kStages];
+  uint64_t kv_ready[kStages];
+  uint64_t kv_empty[kStages];
+  uint64_t s_full[2];
+  uint64_t p_full;
+  uint64_t pv_done;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+struct P1Params {
+  const __nv_bfloat16 *q, *k_cur, *v_cur, *k_prev, *v_prev;
+  const uint8_t *is_seed, *is_new;
+  int L, Hq, Hkv;
+  float scale_log2;
+  __nv_bfloat16* out;
+  float* lse;
+  float* dout_part;
+  uint32_t spin;
+};
+
+__device__ __forceinline__ uint4 ldg16(const void* p) {
+  return *reinterpret_cast<const uint4*>(p);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kP1Threads, 1)
+attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, const P1Params p) {
+  using Lay = P1Layout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  P1Bars* bars = reinterpret_cast<P1Bars*>(smem + Lay::kBar);
+  const uint32_t sbase = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int L = p.L;
+  const int g = h / (p.Hq / p.Hkv);
+  const int q0 = qt * kBM;
+  const int T = (L + kBN - 1) / kBN;
+  volatile int* abort_flag = &bars->abort_flag;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_full, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&bars->kv_full[s], 1);
+      mbar_init(&bars->kv_ready[s], 1);
+      mbar_init(&bars->kv_empty[s], 1);
+    }
+    mbar_init(&bars->s_full[0], 1);
+    mbar_init(&bars->s_full[1], 1);
+    mbar_init(&bars->p_full, 4);
+    mbar_init(&bars->pv_done, 1);
+    mbar_init(&bars->drain, 1);
+    bars->abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  // constant rows of the [1, is_new, 0...] operand: row 0 = ones, rows 2..15 = 0
+  if (warp >= 2) {
+    const int t = threadIdx.x - 64;  // 0..127
+    for (int idx = t; idx < kStages * 2 * 16 * 8; idx += 128) {
+      const int s = idx / (2 * 16 * 8), rem = idx % (2 * 16 * 8);
+      const int ac = rem / (16 * 8), row = (rem / 8) % 16, c = rem % 8;
+      const uint32_t one = 0x3F803F80u;  // two bf16 1.0
+      const uint32_t v = row == 0 ? one : 0u;
+      st_shared_v4(sbase + Lay::kB2 + s * Lay::kB2Bytes + ac * 2048 + sw128(row, c), v, v, v, v);
+    }
+    fence_proxy_async();
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ producer
+    constexpr uint32_t kTxQ = Lay::kTile, kTxKV = 2 * Lay::kTile;
+    if (lane == 0) {
+      mbar_expect_tx(&bars->q_full, kTxQ);
+#pragma unroll
+      for (int ac = 0; ac < D / 64; ++ac)
+        tma_load_4d(smem + Lay::kQ + ac * kAtom, &tmQ, ac * 64, h, q0, b, &bars->q_full);
+    }
+    auto issue = [&](int j) {
+      const int s = j % kStages;
+      if (lane == 0) {
+        mbar_expect_tx(&bars->kv_full[s], kTxKV);
+#pragma unroll
+        for (int ac = 0; ac < D / 64; ++ac) {
+          tma_load_4d(smem + Lay::kK + s * Lay::kTile + ac * kAtom, &tmK, ac * 64, g, j * kBN, b,
+                      &bars->kv_full[s]);
+          tma_load_4d(smem + Lay::kV + s * Lay::kTile + ac * kAtom, &tmV, ac * 64, g, j * kBN, b,
+                      &bars->kv_full[s]);
+        }
+      }
+    };
+    auto finalize = [&](int j) -> bool {
+      const int s = j % kStages;
+      if (!wait_bounded(&bars->kv_full[s], (j / kStages) & 1, p.spin, abort_flag)) return false;
+      const int col0 = j * kBN;
+      // drafting view: seed columns read the step t-1 cache
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const int c = col0 + w * 32 + lane;
+        const bool f = p.is_seed != nullptr && c < L && p.is_seed[(int64_t)b * L + c] != 0;
+        uint32_t bits = __ballot_sync(0xffffffffu, f);
+        while (bits) {
+          const int r = w * 32 + __ffs(bits) - 1;
+          bits &= bits - 1;
+          const int64_t off = (((int64_t)b * L + col0 + r) * p.Hkv + g) * D;
+          const bool is_v = lane >= 16;
+          const int ch = lane & 15;
+          if (ch < D / 8) {
+            const __nv_bfloat16* src = (is_v ? p.v_prev : p.k_prev) + off + ch * 8;
+            const uint4 val = ldg16(src);
+            const uint32_t dst = sbase + (is_v ? Lay::kV : Lay::kK) + s * Lay::kTile +
+                                 (ch / 8) * kAtom + sw128(r, ch & 7);
+            st_shared_v4(dst, val.x, val.y, val.z, val.w);
+          }
+        }
+      }
+      // row 1 of the statistics operand: the tile's newly-written flags
+      if (lane < 16) {
+        uint32_t w4[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int c0 = col0 + lane * 8 + 2 * e;
+          const bool n0 = p.is_new != nullptr && c0 < L && p.is_new[(int64_t)b * L + c0];
+          const bool n1 = p.is_new != nullptr && c0 + 1 < L && p.is_new[(int64_t)b * L + c0 + 1];
+          w4[e] = (n0 ? 0x3F80u : 0u) | (n1 ? 0x3F800000u : 0u);
+        }
+        st_shared_v4(sbase + Lay::kB2 + s * Lay::kB2Bytes + (lane / 8) * 2048 + sw128(1, lane & 7),
+                     w4[0], w4[1], w4[2], w4[3]);
+      }
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->kv_ready[s]);
+      return true;
+    };
+    int issued = 0, finalized = 0;
+    for (int j = 0; j < T && j < kStages; ++j) { issue(j); ++issued; }
+    bool ok = finalize(0);
+    if (ok) finalized = 1;
+    for (int j = 0; ok && j < T; ++j) {
+      if (j + 1 < T) {
+        ok = finalize(j + 1);
+        if (!ok) break;
+        finalized = j + 2;
+      }
+      if (j + kStages < T) {
+        ok = wait_bounded(&bars->kv_empty[j % kStages], (j / kStages) & 1, p.spin, abort_flag);
+        if (!ok) break;
+        issue(j + kStages);
+        ++issued;
+      }
+    }
+    // never leave with TMA writes in flight
+    for (int j = finalized; j < issued; ++j)
+      wait_bounded(&bars->kv_full[j % kStages], (j / kStages) & 1, p.spin, abort_flag);
+    wait_bounded(&bars->q_full, 0, p.spin, abort_flag);
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idS = idesc_bf16(kBM, kBN, false);
+      const uint32_t idO = idesc_bf16(kBM, D, true);
+      const uint32_t idSt = idesc_bf16(kBM, 16, false);
+      const uint32_t sQ = sbase + Lay::kQ;
+      auto qk = [&](int j) {
+        const int s = j % kStages;
+        const uint32_t sK = sbase + Lay::kK + s * Lay::kTile;
+        const uint32_t dS = tmem + ((j & 1) ? Lay::kS1 : Lay::kS0);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * kAtom + (kk % 4) * 32;
+          mma_bf16(dS, desc_kmajor_sw128(sQ + off), desc_kmajor_sw128(sK + off), idS, kk > 0);
+        }
+        mma_commit(&bars->s_full[j & 1]);
+      };
+      bool ok = wait_bounded(&bars->q_full, 0, p.spin, abort_flag);
+      ok = ok && wait_bounded(&bars->kv_ready[0], 0, p.spin, abort_flag);
+      if (ok) {
+        fence_after_sync();
+        qk(0);
+      }
+      for (int j = 0; ok && j < T; ++j) {
+        if (j + 1 < T) {
+          const int s1 = (j + 1) % kStages;
+          ok = wait_bounded(&bars->kv_ready[s1], ((j + 1) / kStages) & 1, p.spin, abort_flag);
+          if (!ok) break;
+          fence_after_sync();
+          qk(j + 1);
+        }
+        ok = wait_bounded(&bars->p_full, j & 1, p.spin, abort_flag);
+        if (!ok) break;
+        fence_after_sync();
+        const int s = j % kStages;
+        const uint32_t sP = sbase + Lay::kP;
+        const uint32_t sV = sbase + Lay::kV + s * Lay::kTile;
+        const uint32_t sB2 = sbase + Lay::kB2 + s * Lay::kB2Bytes;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          const uint64_t a = desc_kmajor_sw128(sP + (kk / 4) * kAtom + (kk % 4) * 32);
+          const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
+          mma_bf16(tmem + Lay::kO, a, desc_mnmajor_sw128(sV + kk * 16 * 128, kAtom), idO, acc);
+          mma_bf16(tmem + Lay::kSt, a, desc_kmajor_sw128(sB2 + (kk / 4) * 2048 + (kk % 4) * 32),
+                   idSt, acc);
+        }
+        mma_commit(&bars->pv_done);
+        mma_commit(&bars->kv_empty[s]);
+      }
+      // all issued tensor-core work done before TMEM is released
+      mma_commit(&bars->drain);
+      wait_bounded(&bars->drain, 0, p.spin, abort_flag);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------------ softmax
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const int i = q0 + r;
+    const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
+    const bool seed_row =
+        i < L && p.is_seed != nullptr && p.is_seed[(int64_t)b * L + i] != 0;
+    const float c2 = p.scale_log2;
+    float m = -INFINITY;
+    bool ok = true;
+    const uint32_t sP = sbase + Lay::kP;
+    for (int j = 0; j < T; ++j) {
+      ok = wait_bounded(&bars->s_full[j & 1], (j >> 1) & 1, p.spin, abort_flag);
+      if (!ok) break;
+      fence_after_sync();
+      float s[kBN];
+      {
+        const uint32_t scol = (j & 1) ? Lay::kS1 : Lay::kS0;
+#pragma unroll
+        for (int q = 0; q < kBN / 32; ++q) {
+          float t[32];
+          tmem_ld32(tl + scol + q * 32, t);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) s[q * 32 + e] = t[e];
+        }
+        tmem_wait_ld();
+      }
+      if ((j + 1) * kBN > L) {
+#pragma unroll
+        for (int c = 0; c < kBN; ++c)
+          if (j * kBN + c >= L) s[c] = -INFINITY;
+      }
+      if (seed_row && j == qt) {
+#pragma unroll
+        for (int c = 0; c < kBN; ++c)
+          if (c == r) s[c] = -INFINITY;
+      }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < kBN; ++c) mx = fmaxf(mx, s[c]);
+      mx *= c2;
+      const bool need = mx > m + 8.f;
+      const float m_new = need ? mx : m;
+      if (j > 0) {
+        ok = wait_bounded(&bars->pv_done, (j - 1) & 1, p.spin, abort_flag);
+        if (!ok) break;
+        fence_after_sync();
+      }
+      const bool resc = need && j > 0 && m != -INFINITY;
+      if (__any_sync(0xffffffffu, resc)) {
+        const float f = resc ? exp2f(m - m_new) : 1.f;
+#pragma unroll 1
+        for (int q = 0; q < D / 32 + 1; ++q) {
+          float o[32];
+          tmem_ld32(tl + Lay::kO + q * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] *= f;
+          tmem_st32(tl + Lay::kO + q * 32, o);
+        }
+        tmem_wait_st();
+      }
+      m = m_new;
+      const bool live = m != -INFINITY;
+#pragma unroll
+      for (int cc = 0; cc < kBN / 8; ++cc) {
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float a = live ? exp2f(fmaf(s[cc * 8 + 2 * e], c2, -m)) : 0.f;
+          const float bb = live ? exp2f(fmaf(s[cc * 8 + 2 * e + 1], c2, -m)) : 0.f;
+          w[e] = pack_bf16(a, bb);
+        }
+        st_shared_v4(sP + (cc / 8) * kAtom + sw128(r, cc & 7), w[0], w[1], w[2], w[3]);
+      }
+      fence_proxy_async();
+      fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->p_full);
+    }
+    if (ok) ok = wait_bounded(&bars->pv_done, (T - 1) & 1, p.spin, abort_flag);
+    if (ok) {
+      fence_after_sync();
+      float o[D];
+#pragma unroll
+      for (int q = 0; q < D / 32; ++q) {
+        float t[32];
+        tmem_ld32(tl + Lay::kO + q * 32, t);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[q * 32 + e] = t[e];
+      }
+      float st[32];
+      tmem_ld32(tl + Lay::kSt, st);
+      tmem_wait_ld();
+      float l = st[0], ln = st[1];
+      if (seed_row) {
+        // leave-one-out diagonal: the seed's own column from the masked input
+        const int64_t qoff = (((int64_t)b * L + i) * p.Hq + h) * D;
+        const int64_t koff = (((int64_t)b * L + i) * p.Hkv + g) * D;
+        float dot = 0.f;
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) {
+          const uint4 qa = ldg16(p.q + qoff + c * 8), ka = ldg16(p.k_cur + koff + c * 8);
+          dot += bf16lo(qa.x) * bf16lo(ka.x) + bf16hi(qa.x) * bf16hi(ka.x) +
+                 bf16lo(qa.y) * bf16lo(ka.y) + bf16hi(qa.y) * bf16hi(ka.y) +
+                 bf16lo(qa.z) * bf16lo(ka.z) + bf16hi(qa.z) * bf16hi(ka.z) +
+                 bf16lo(qa.w) * bf16lo(ka.w) + bf16hi(qa.w) * bf16hi(ka.w);
+        }
+        const float sd = dot * c2;
+        const float mn = fmaxf(m, sd);
+        const float f = m == -INFINITY ? 0.f : exp2f(m - mn);
+        const float pd = exp2f(sd - mn);
+        const bool self_new = p.is_new != nullptr && p.is_new[(int64_t)b * L + i] != 0;
+        l = l * f + pd;
+        ln = ln * f + (self_new ? pd : 0.f);
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) {
+          const uint4 va = ldg16(p.v_cur + koff + c * 8);
+          o[c * 8 + 0] = fmaf(pd, bf16lo(va.x), o[c * 8 + 0] * f);
+          o[c * 8 + 1] = fmaf(pd, bf16hi(va.x), o[c * 8 + 1] * f);
+          o[c * 8 + 2] = fmaf(pd, bf16lo(va.y), o[c * 8 + 2] * f);
+          o[c * 8 + 3] = fmaf(pd, bf16hi(va.y), o[c * 8 + 3] * f);
+          o[c * 8 + 4] = fmaf(pd, bf16lo(va.z), o[c * 8 + 4] * f);
+          o[c * 8 + 5] = fmaf(pd, bf16hi(va.z), o[c * 8 + 5] * f);
+          o[c * 8 + 6] = fmaf(pd, bf16lo(va.w), o[c * 8 + 6] * f);
+          o[c * 8 + 7] = fmaf(pd, bf16hi(va.w), o[c * 8 + 7] * f);
+        }
+        m = mn;
+      }
+      if (i < L) {
+        const float inv = 1.f / l;
+        uint4* dst = reinterpret_cast<uint4*>(p.out + (((int64_t)b * L + i) * p.Hq + h) * D);
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) {
+          uint4 v;
+          v.x = pack_bf16(o[c * 8 + 0] * inv, o[c * 8 + 1] * inv);
+          v.y = pack_bf16(o[c * 8 + 2] * inv, o[c * 8 + 3] * inv);
+          v.z = pack_bf16(o[c * 8 + 4] * inv, o[c * 8 + 5] * inv);
+          v.w = pack_bf16(o[c * 8 + 6] * inv, o[c * 8 + 7] * inv);
+          dst[c] = v;
+        }
+        p.lse[((int64_t)b * p.Hq + h) * L + i] = (m + log2f(l)) * kLn2;
+        if (p.dout_part) p.dout_part[((int64_t)b * p.Hq + h) * L + i] = ln * inv;
+      }
+    }
+  }
+  fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    fence_after_sync();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// --------------------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return (PFN_cuTensorMapEncodeTiled_v12000) nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }();
+  return fn;
+}
+
+// 4-D map over a [B, L, H, D] bf16 tensor, dims innermost first {D, H, L, B};
+// box = 64 head-dim elements (128 bytes) x 1 head x 128 positions x 1 sequence.
+bool make_map(CUtensorMap* map, const void* base, int D, int H, int L, int B) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)L, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)L * H * D * 2};
+  cuuint32_t box[4] = {64, 1, 128, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D>
+cudaError_t launch_p1(const AttnArgs& a, cudaStream_t stream) {
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, a.q, D, a.Hq, a.L, a.B) || !make_map(&tk, a.k_cur, D, a.Hkv, a.L, a.B) ||
+      !make_map(&tv, a.v_cur, D, a.Hkv, a.L, a.B))
+    return cudaErrorInvalidValue;
+  const int smem = P1Layout<D>::kBytes + 1024;
+  static int configured[64] = {};
+  const int dev = device_info().device;
+  if (!configured[dev & 63]) {
+    cudaError_t e = cudaFuncSetAttribute(attn_p1_kernel<D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    configured[dev & 63] = 1;
+  }
+  P1Params p;
+  p.q = static_cast<const __nv_bfloat16*>(a.q);
+  p.k_cur = static_cast<const __nv_bfloat16*>(a.k_cur);
+  p.v_cur = static_cast<const __nv_bfloat16*>(a.v_cur);
+  p.k_prev = static_cast<const __nv_bfloat16*>(a.k_prev);
+  p.v_prev = static_cast<const __nv_bfloat16*>(a.v_prev);
+  p.is_seed = a.is_seed;
+  p.is_new = a.is_new;
+  p.L = a.L;
+  p.Hq = a.Hq;
+  p.Hkv = a.Hkv;
+  p.scale_log2 = a.scale * kLog2e;
+  p.out = static_cast<__nv_bfloat16*>(a.out);
+  p.lse = a.lse;
+  p.dout_part = a.dout_part;
+  p.spin = spin_limit();
+  dim3 grid((a.L + kBM - 1) / kBM, a.Hq, a.B);
+  attn_p1_kernel<D><<<grid, kP1Threads, smem, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+// Pass 1 on tensor cores; pass 2 (d_in) still on CUDA cores.
+cudaError_t launch_simt_pass2_bf16(const AttnArgs& a, cudaStream_t stream);
+
 cudaError_t launch_attention_tc(const AttnArgs& a, cudaStream_t stream, bool* handled) {
-  (void)a;
-  (void)stream;
-  *handled = false;
-  return cudaSuccess;
+  *handled = true;
+  cudaError_t err = a.d == 64 ? launch_p1<64>(a, stream) : launch_p1<128>(a, stream);
+  if (err != cudaSuccess) return err;
+  if (a.d_in && a.is_masked) err = launch_simt_pass2_bf16(a, stream);
+  return err;
 }
 
 }  // namespace dd
