@@ -337,16 +337,8 @@ cudaError_t launch_simt(const AttnArgs& a, cudaStream_t stream) {
 
 }  // namespace
 
-cudaError_t launch_simt_pass2_bf16(const AttnArgs& a, cudaStream_t stream) {
-  dim3 g2((a.L + kCols - 1) / kCols, a.Hq, a.B);
-  if (a.d == 64)
-    simt_pass2_kernel<__nv_bfloat16, 64><<<g2, 128, 0, stream>>>(a);
-  else
-    simt_pass2_kernel<__nv_bfloat16, 128><<<g2, 128, 0, stream>>>(a);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_attention_tc(const AttnArgs& a, cudaStream_t stream, bool* handled);
+cudaError_t launch_attention_tc(const AttnArgs& a, cudaStream_t stream, bool* handled,
+                                int* din_slices);
 
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t stream) {
   cudaError_t err;
@@ -356,8 +348,9 @@ cudaError_t launch_attention(const AttnArgs& a, cudaStream_t stream) {
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
   }
   bool handled = false;
+  int din_slices = a.Hq;  // d_in partials: per query head (CUDA-core pass 2) or per kv head
   if (a.dtype == DD_BF16) {
-    err = launch_attention_tc(a, stream, &handled);
+    err = launch_attention_tc(a, stream, &handled, &din_slices);
     if (err != cudaSuccess) return err;
   }
   if (!handled) {
@@ -381,7 +374,7 @@ cudaError_t launch_attention(const AttnArgs& a, cudaStream_t stream) {
   }
   if (a.d_in) {
     if (need_din) {
-      head_reduce_kernel<<<grid, 256, 0, stream>>>(a.din_part, a.Hq, a.L, 1.f / a.Hq,
+      head_reduce_kernel<<<grid, 256, 0, stream>>>(a.din_part, din_slices, a.L, 1.f / a.Hq,
                                                    a.accumulate, total, a.d_in);
     } else if (!a.accumulate) {
       cudaMemsetAsync(a.d_in, 0, total * sizeof(float), stream);

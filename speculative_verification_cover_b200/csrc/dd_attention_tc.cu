@@ -429,6 +429,220 @@ attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   }
 }
 
+// --------------------------------------------------------------------------- pass 2
+// d_in partials: one CTA per (128 key columns, kv head, sequence). The key tile
+// (drafting view: seed columns from the cache) stays in shared memory; the CTA
+// loops over the G query heads sharing this kv head and over tiles of 128
+// still-masked query rows (gathered). S^T = K Q_m^T puts one key column per
+// TMEM lane, so each consumer thread sums exp2(S * scale * log2e - lse2) over
+// its own column without any cross-thread reduction.
+//   warps 0-3  producers: warp 0 issues the key TMA and patches seed rows; all
+//              four gather masked query rows (plain loads, swizzled stores) and
+//              their lse (natural log -> log2 units) into a double buffer
+//   warp 4     MMA issuer
+//   warps 5-8  consumers (one key column each)
+constexpr int kP2Threads = 288;
+
+template <int D>
+struct P2Layout {
+  static constexpr int kTile = (D / 64) * kAtom;
+  static constexpr int kK = 0;
+  static constexpr int kQ = kK + kTile;               // two buffers
+  static constexpr int kLse = kQ + 2 * kTile;         // two buffers of 128 floats
+  static constexpr int kBar = kLse + 2 * 128 * 4;
+  static constexpr int kBytes = kBar + 256;
+};
+
+struct P2Bars {
+  uint64_t k_full, k_ready;
+  uint64_t q_full[2];
+  uint64_t s_full[2];
+  uint64_t c_done[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+struct P2Params {
+  const __nv_bfloat16 *q, *k_prev;
+  const uint8_t* is_seed;
+  const float* lse;
+  const int32_t *mrows, *mcount;
+  int L, Hq, Hkv;
+  float scale_log2;
+  float* din_part;  // [B, Hkv, L]
+  uint32_t spin;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kP2Threads, 1)
+attn_p2_kernel(const __grid_constant__ CUtensorMap tmK, const P2Params p) {
+  using Lay = P2Layout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  P2Bars* bars = reinterpret_cast<P2Bars*>(smem + Lay::kBar);
+  const uint32_t sbase = smem_u32(smem);
+  float* lse2 = reinterpret_cast<float*>(smem + Lay::kLse);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kt = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int L = p.L;
+  const int G = p.Hq / p.Hkv;
+  const int col0 = kt * kBN;
+  const int M = p.mcount[b];
+  const int nrt = (M + 127) / 128;
+  const int NT = G * nrt;
+  volatile int* abort_flag = &bars->abort_flag;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->k_full, 1);
+    mbar_init(&bars->k_ready, 1);
+    for (int u = 0; u < 2; ++u) {
+      mbar_init(&bars->q_full[u], 128);
+      mbar_init(&bars->s_full[u], 1);
+      mbar_init(&bars->c_done[u], 4);
+    }
+    mbar_init(&bars->drain, 1);
+    bars->abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 4) {
+    tmem_alloc(&bars->tmem_base, 256);
+    tmem_relinquish();
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp < 4) {
+    // ------------------------------------------------------------------ producers
+    const int pt = threadIdx.x;  // 0..127: the masked row this thread gathers
+    if (warp == 0) {
+      if (lane == 0) {
+        mbar_expect_tx(&bars->k_full, Lay::kTile);
+#pragma unroll
+        for (int ac = 0; ac < D / 64; ++ac)
+          tma_load_4d(smem + Lay::kK + ac * kAtom, &tmK, ac * 64, g, col0, b, &bars->k_full);
+      }
+      if (wait_bounded(&bars->k_full, 0, p.spin, abort_flag)) {
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          const int c = col0 + w * 32 + lane;
+          const bool f = p.is_seed != nullptr && c < L && p.is_seed[(int64_t)b * L + c] != 0;
+          uint32_t bits = __ballot_sync(0xffffffffu, f);
+          while (bits) {
+            const int r = w * 32 + __ffs(bits) - 1;
+            bits &= bits - 1;
+            if (lane < D / 8) {
+              const uint4 val =
+                  ldg16(p.k_prev + (((int64_t)b * L + col0 + r) * p.Hkv + g) * D + lane * 8);
+              st_shared_v4(sbase + Lay::kK + (lane / 8) * kAtom + sw128(r, lane & 7), val.x,
+                           val.y, val.z, val.w);
+            }
+          }
+        }
+        fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->k_ready);
+      }
+    }
+    for (int t = 0; t < NT; ++t) {
+      const int u = t & 1;
+      if (t >= 2 && !wait_bounded(&bars->c_done[u], ((t >> 1) - 1) & 1, p.spin, abort_flag)) break;
+      const int hh = g * G + t / nrt;
+      const int m = (t % nrt) * 128 + pt;
+      const uint32_t qb = sbase + Lay::kQ + u * Lay::kTile;
+      if (m < M) {
+        const int pos = p.mrows[(int64_t)b * L + m];
+        const __nv_bfloat16* src = p.q + (((int64_t)b * L + pos) * p.Hq + hh) * D;
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) {
+          const uint4 val = ldg16(src + c * 8);
+          st_shared_v4(qb + (c / 8) * kAtom + sw128(pt, c & 7), val.x, val.y, val.z, val.w);
+        }
+        lse2[u * 128 + pt] = p.lse[((int64_t)b * p.Hq + hh) * L + pos] * kLog2e;
+      } else {
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c)
+          st_shared_v4(qb + (c / 8) * kAtom + sw128(pt, c & 7), 0u, 0u, 0u, 0u);
+        lse2[u * 128 + pt] = INFINITY;
+      }
+      fence_proxy_async();
+      mbar_arrive(&bars->q_full[u]);
+    }
+  } else if (warp == 4) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idS = idesc_bf16(kBM, kBN, false);
+      const uint32_t sK = sbase + Lay::kK;
+      bool ok = NT == 0 || wait_bounded(&bars->k_ready, 0, p.spin, abort_flag);
+      for (int t = 0; ok && t < NT; ++t) {
+        const int u = t & 1;
+        ok = wait_bounded(&bars->q_full[u], (t >> 1) & 1, p.spin, abort_flag);
+        if (ok && t >= 2) ok = wait_bounded(&bars->c_done[u], ((t >> 1) - 1) & 1, p.spin, abort_flag);
+        if (!ok) break;
+        fence_after_sync();
+        const uint32_t sQ = sbase + Lay::kQ + u * Lay::kTile;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * kAtom + (kk % 4) * 32;
+          mma_bf16(tmem + u * 128, desc_kmajor_sw128(sK + off), desc_kmajor_sw128(sQ + off), idS,
+                   kk > 0);
+        }
+        mma_commit(&bars->s_full[u]);
+      }
+      mma_commit(&bars->drain);
+      wait_bounded(&bars->drain, 0, p.spin, abort_flag);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------------ consumers
+    const int quarter = warp & 3;
+    const int j = quarter * 32 + lane;  // key column within the tile
+    const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
+    const float c2 = p.scale_log2;
+    float acc = 0.f;
+    bool ok = true;
+    for (int t = 0; t < NT; ++t) {
+      const int u = t & 1;
+      ok = wait_bounded(&bars->s_full[u], (t >> 1) & 1, p.spin, abort_flag);
+      if (!ok) break;
+      fence_after_sync();
+      float s[kBN];
+#pragma unroll
+      for (int q = 0; q < kBN / 32; ++q) {
+        float tt[32];
+        tmem_ld32(tl + u * 128 + q * 32, tt);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) s[q * 32 + e] = tt[e];
+      }
+      tmem_wait_ld();
+      const float4* lv = reinterpret_cast<const float4*>(lse2 + u * 128);
+      float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+      for (int c4 = 0; c4 < kBN / 4; ++c4) {
+        const float4 l4 = lv[c4];
+        a0 += exp2f(fmaf(s[4 * c4 + 0], c2, -l4.x));
+        a1 += exp2f(fmaf(s[4 * c4 + 1], c2, -l4.y));
+        a0 += exp2f(fmaf(s[4 * c4 + 2], c2, -l4.z));
+        a1 += exp2f(fmaf(s[4 * c4 + 3], c2, -l4.w));
+      }
+      acc += a0 + a1;
+      fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->c_done[u]);
+    }
+    if (col0 + j < L) p.din_part[((int64_t)b * p.Hkv + g) * L + col0 + j] = acc;
+  }
+  fence_before_sync();
+  __syncthreads();
+  if (warp == 4) {
+    fence_after_sync();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
 // --------------------------------------------------------------------------- host side
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
@@ -493,16 +707,49 @@ cudaError_t launch_p1(const AttnArgs& a, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+template <int D>
+cudaError_t launch_p2(const AttnArgs& a, cudaStream_t stream) {
+  CUtensorMap tk;
+  if (!make_map(&tk, a.k_cur, D, a.Hkv, a.L, a.B)) return cudaErrorInvalidValue;
+  const int smem = P2Layout<D>::kBytes + 1024;
+  static int configured[64] = {};
+  const int dev = device_info().device;
+  if (!configured[dev & 63]) {
+    cudaError_t e = cudaFuncSetAttribute(attn_p2_kernel<D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    configured[dev & 63] = 1;
+  }
+  P2Params p;
+  p.q = static_cast<const __nv_bfloat16*>(a.q);
+  p.k_prev = static_cast<const __nv_bfloat16*>(a.k_prev);
+  p.is_seed = a.is_seed;
+  p.lse = a.lse;
+  p.mrows = a.mrows;
+  p.mcount = a.mcount;
+  p.L = a.L;
+  p.Hq = a.Hq;
+  p.Hkv = a.Hkv;
+  p.scale_log2 = a.scale * kLog2e;
+  p.din_part = a.din_part;
+  p.spin = spin_limit();
+  dim3 grid((a.L + kBN - 1) / kBN, a.Hkv, a.B);
+  attn_p2_kernel<D><<<grid, kP2Threads, smem, stream>>>(tk, p);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
-// Pass 1 on tensor cores; pass 2 (d_in) still on CUDA cores.
-cudaError_t launch_simt_pass2_bf16(const AttnArgs& a, cudaStream_t stream);
-
-cudaError_t launch_attention_tc(const AttnArgs& a, cudaStream_t stream, bool* handled) {
+// Both passes on tensor cores. d_in partials are per kv head ([B, Hkv, L]).
+cudaError_t launch_attention_tc(const AttnArgs& a, cudaStream_t stream, bool* handled,
+                                int* din_slices) {
   *handled = true;
   cudaError_t err = a.d == 64 ? launch_p1<64>(a, stream) : launch_p1<128>(a, stream);
   if (err != cudaSuccess) return err;
-  if (a.d_in && a.is_masked) err = launch_simt_pass2_bf16(a, stream);
+  if (a.d_in && a.is_masked) {
+    err = a.d == 64 ? launch_p2<64>(a, stream) : launch_p2<128>(a, stream);
+    *din_slices = a.Hkv;
+  }
   return err;
 }
 
