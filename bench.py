@@ -52,15 +52,17 @@ def parse():
     p.add_argument("--steps", type=int, default=1000)
     p.add_argument("--warmup", type=int, default=50)
     p.add_argument("--workload", default=W.LLADA8B_L512.name)
+    p.add_argument("--batch", type=int, default=0, help="override the workload's batch size")
     p.add_argument("--impl", choices=("ours", "reference"), default="ours")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     return p.parse_args()
 
 
-def spec_by_name(name):
+def spec_by_name(name, batch=0):
     for s in W.WORKLOADS:
         if s.name == name or s.name.startswith(name):
-            return s
+            return s.replace(B=batch) if batch > 0 else s
     raise SystemExit(f"unknown workload {name}")
 
 
@@ -261,7 +263,7 @@ def run_reference(args, world, rank):
     """The oracle as the reference arm: bounded samples of the same workload per step."""
     if rank != 0:
         return
-    spec = spec_by_name(args.workload)
+    spec = spec_by_name(args.workload, args.batch)
     x = W.make_inputs(spec, "cpu", seed=shard_seed(spec, 0))
     # Per-step sample sized so the whole run takes ~90 s of host time: every
     # hs-th head and every rs-th verified row of one sequence, select/decide whole.
@@ -297,11 +299,43 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def run_e2e(step, x, K, world):
+    """Steps through the public API from pinned host buffers: host->device copy of every
+    input, the step, device->host copy of the decisions, all inside the timed window."""
+    from speculative_verification_cover_b200.step import INPUT_KEYS
+    mean = lambda v: float(np.mean(v))
+    host = {k: x[k].detach().cpu().pin_memory() for k in INPUT_KEYS}
+
+    outs = step.result_tensors()
+    host_out = [t.detach().cpu().pin_memory() for t in outs]
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+    Ke = max(3, min(K, 50))
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(Ke)]
+    for k in range(Ke + 2):
+        e = e2e_ev[k - 2] if k >= 2 else None
+        if e:
+            e[0].record()
+        for key in INPUT_KEYS:
+            step.x[key].copy_(host[key], non_blocking=True)
+        step.replay()
+        for t, h in zip(outs, host_out):
+            h.copy_(t, non_blocking=True)
+        if e:
+            e[1].record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks([mean([a.elapsed_time(b) for a, b in e2e_ev])], world)[0]
+
+    return {"value": world * 1000.0 / e2e_ms, "unit": "steps/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h}
+
+
 def run_ours(args, world, rank, local):
     from speculative_verification_cover_b200 import dd
     from speculative_verification_cover_b200.step import INPUT_KEYS, KERNELS_PER_STEP, VerifyStep
     dd.lib()  # fail loudly if the library is missing
-    spec = spec_by_name(args.workload)
+    spec = spec_by_name(args.workload, args.batch)
     dev = torch.device("cuda", local)
     x = W.make_inputs(spec, dev, seed=shard_seed(spec, rank))
     step = VerifyStep(spec, x)
@@ -334,28 +368,7 @@ def run_ours(args, world, rank, local):
     assert dd.dd_get_device_error() == dd.DD_OK
 
     # ---- end to end through the public API: pinned host inputs -> device -> host decisions
-    host = {k: x[k].detach().cpu().pin_memory() for k in INPUT_KEYS}
-    outs = step.result_tensors()
-    host_out = [t.detach().cpu().pin_memory() for t in outs]
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = sum(t.numel() * t.element_size() for t in host_out)
-    Ke = max(3, min(K, 50))
-    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(Ke)]
-    for k in range(Ke + 2):
-        e = e2e_ev[k - 2] if k >= 2 else None
-        if e:
-            e[0].record()
-        for key in INPUT_KEYS:
-            step.x[key].copy_(host[key], non_blocking=True)
-        step.replay()
-        for t, h in zip(outs, host_out):
-            h.copy_(t, non_blocking=True)
-        if e:
-            e[1].record()
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks([mean([a.elapsed_time(b) for a, b in e2e_ev])], world)[0]
-
+    e2e = None if args.no_e2e else run_e2e(step, x, K, world)
     hbm, bf16, bf16_s, peak_src = peaks()
     vbytes, aflops, pflops = algorithmic(spec)
     achieved = vbytes / (v_ms * 1e-3) / 1e9
@@ -384,8 +397,7 @@ def run_ours(args, world, rank, local):
                       "achieved_tflops": (aflops + pflops) / (a_ms * 1e-3) / 1e12,
                       "peak_tflops": bf16, "frac": (aflops + pflops) / (a_ms * 1e-3) / 1e12 / bf16,
                       "peak_source": f"MEASURED_PEAKS.json bf16_tflops ({peak_src})"},
-        "e2e": {"value": world * 1000.0 / e2e_ms, "unit": "steps/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
+        "e2e": e2e,
         "gpu_launches": KERNELS_PER_STEP * K,
         "clocks": clocks.summary(),
     }

@@ -96,12 +96,15 @@ enum { DD_NONE = 0, DD_KEEP = 1, DD_REPLACE = 2, DD_REMASK = 3 };
  * out               [B,L,Hq,d] same dtype as q (required)
  * lse               [B,Hq,L] fp32 natural-log LSE (required)
  * d_in, d_out       [B,L] fp32, each may be NULL to skip it
- * workspace         device scratch of at least
+ * workspace         device scratch (required) of at least
  *                   dd_dualview_attention_workspace_size(B,L,Hq,Hkv,d) bytes,
- *                   256-byte aligned; contents on entry are ignored.
+ *                   256-byte aligned; contents on entry are ignored. Calls that
+ *                   share a workspace must not overlap on the GPU.
+ * Preconditions: is_seed and is_masked are disjoint (seeds are previously
+ * unmasked tokens); K/V/Q values are finite.
  * Errors: DD_ERR_INVALID_ARG for null required pointers, non-positive sizes,
  * Hq % Hkv != 0, misalignment or a short workspace; DD_ERR_UNSUPPORTED for
- * d not in {64,128}.
+ * d not in {64,128}, or L > 32768 with DD_BF16.
  */
 dd_status dd_dualview_attention(
     const void* q, const void* k_cur, const void* v_cur,
@@ -146,15 +149,24 @@ typedef struct {
  *                       word = Philox4x32-10 output word (v & 3),
  *                       U = (2*(word >> 9) + 1) * 2^-24,  g = -ln(-ln U)
  * Statistics (lse, conf, entropy, kl) use the T = 1 distributions.
- * Ties in argmax / samples go to the lowest vocabulary index.
- * Errors: DD_ERR_INVALID_ARG for null logits, B/R/V < 1, ld < V, temperature
- * < 0, misaligned logits or ld.
+ * Ties in argmax / samples go to the lowest vocabulary index. Logits must be
+ * finite.
+ * workspace           device scratch (required) of at least
+ *                     dd_verify_logits_workspace_size(B,R,V,dtype) bytes, 256-byte
+ *                     aligned; holds per-row partial states; contents on entry are
+ *                     ignored. Calls sharing a workspace must not overlap on the GPU.
+ * Errors: DD_ERR_INVALID_ARG for null logits/out/workspace, B/R/V < 1, ld < V,
+ * temperature < 0, misaligned logits or ld, a short workspace.
  */
 dd_status dd_verify_logits(
     const void* logits_t, const void* logits_d, dd_dtype dtype,
     int B, int R, int V, int64_t ld, int pos_offset,
     float temperature, uint64_t seed, uint64_t step,
-    const dd_row_stats* out, void* stream);
+    const dd_row_stats* out, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of device scratch dd_verify_logits needs (0 on invalid sizes). Pure host
+ * function; the bound holds on any device. */
+size_t dd_verify_logits_workspace_size(int B, int R, int V, dd_dtype dtype);
 
 /*
  * dd_coupled_gumbel -- write the shared Gumbel noise g[b, r, v] (fp32, row

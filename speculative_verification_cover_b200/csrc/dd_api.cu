@@ -85,12 +85,10 @@ dd_status dd_dualview_attention(const void* q, const void* k_cur, const void* v_
   if (!aligned16(q) || !aligned16(k_cur) || !aligned16(v_cur) || !aligned16(out) ||
       (k_prev && !aligned16(k_prev)) || (v_prev && !aligned16(v_prev)))
     return DD_ERR_INVALID_ARG;
-  const bool need_ws = (d_in && is_masked) || (d_out && is_new);
+  if (dtype == DD_BF16 && L > kTcMaxL) return DD_ERR_UNSUPPORTED;
   const AttnWorkspace ws = attn_workspace_layout(B, L, Hq);
-  if (need_ws) {
-    if (!workspace || workspace_bytes < ws.total) return DD_ERR_INVALID_ARG;
-    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return DD_ERR_INVALID_ARG;
-  }
+  if (!workspace || workspace_bytes < ws.total) return DD_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return DD_ERR_INVALID_ARG;
   AttnArgs a{};
   a.q = q; a.k_cur = k_cur; a.v_cur = v_cur; a.k_prev = k_prev; a.v_prev = v_prev;
   a.is_seed = is_seed; a.is_masked = is_masked; a.is_new = is_new;
@@ -100,16 +98,25 @@ dd_status dd_dualview_attention(const void* q, const void* k_cur, const void* v_
   a.accumulate = accumulate_stats ? 1 : 0;
   a.out = out; a.lse = lse; a.d_in = d_in; a.d_out = d_out;
   char* w = static_cast<char*>(workspace);
-  a.dout_part = need_ws ? reinterpret_cast<float*>(w + ws.dout_off) : nullptr;
-  a.din_part = need_ws ? reinterpret_cast<float*>(w + ws.din_off) : nullptr;
-  a.mrows = need_ws ? reinterpret_cast<int32_t*>(w + ws.mrows_off) : nullptr;
-  a.mcount = need_ws ? reinterpret_cast<int32_t*>(w + ws.mcount_off) : nullptr;
+  a.dout_part = reinterpret_cast<float*>(w + ws.dout_off);
+  a.din_part = reinterpret_cast<float*>(w + ws.din_off);
+  a.mrows = reinterpret_cast<int32_t*>(w + ws.mrows_off);
+  a.mcount = reinterpret_cast<int32_t*>(w + ws.mcount_off);
+  a.seedbits = reinterpret_cast<uint32_t*>(w + ws.seedbits_off);
+  a.newbits = reinterpret_cast<uint32_t*>(w + ws.newbits_off);
   return from_cuda(launch_attention(a, static_cast<cudaStream_t>(stream)));
+}
+
+size_t dd_verify_logits_workspace_size(int B, int R, int V, dd_dtype dtype) {
+  if (B < 1 || R < 1 || V < 1 || !valid_dtype(dtype)) return 0;
+  if ((int64_t)B * R > (1ll << 27)) return 0;
+  return verify_workspace_bytes(B, R, V, dtype);
 }
 
 dd_status dd_verify_logits(const void* logits_t, const void* logits_d, dd_dtype dtype, int B,
                            int R, int V, int64_t ld, int pos_offset, float temperature,
-                           uint64_t seed, uint64_t step, const dd_row_stats* out, void* stream) {
+                           uint64_t seed, uint64_t step, const dd_row_stats* out,
+                           void* workspace, size_t workspace_bytes, void* stream) {
   if (!logits_t || !logits_d || !out) return DD_ERR_INVALID_ARG;
   if (!valid_dtype(dtype)) return DD_ERR_INVALID_ARG;
   if (B < 1 || R < 1 || V < 1 || ld < V || pos_offset < 0) return DD_ERR_INVALID_ARG;
@@ -117,8 +124,11 @@ dd_status dd_verify_logits(const void* logits_t, const void* logits_d, dd_dtype 
   if (!(temperature >= 0.f) || isinf(temperature)) return DD_ERR_INVALID_ARG;
   if (!aligned16(logits_t) || !aligned16(logits_d)) return DD_ERR_INVALID_ARG;
   if ((ld * (int64_t)elem_size(dtype)) % 16 != 0) return DD_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < verify_workspace_bytes(B, R, V, dtype))
+    return DD_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return DD_ERR_INVALID_ARG;
   return from_cuda(launch_verify_logits(logits_t, logits_d, dtype, B, R, V, ld, pos_offset,
-                                        temperature, seed, step, *out,
+                                        temperature, seed, step, *out, workspace,
                                         static_cast<cudaStream_t>(stream)));
 }
 

@@ -24,18 +24,38 @@ AttnWorkspace attn_workspace_layout(int B, int L, int Hq) {
   w.din_off = up(w.dout_off + part);
   w.mrows_off = up(w.din_off + part);
   w.mcount_off = up(w.mrows_off + (size_t)B * L * sizeof(int32_t));
-  w.total = up(w.mcount_off + (size_t)B * sizeof(int32_t));
+  const size_t words = (size_t)B * ((L + 31) / 32) * sizeof(uint32_t);
+  w.seedbits_off = up(w.mcount_off + (size_t)B * sizeof(int32_t));
+  w.newbits_off = up(w.seedbits_off + words);
+  w.total = up(w.newbits_off + words);
   return w;
 }
 
 namespace {
 
 // ---------------------------------------------------------------------------
-// Masked query rows of each sequence, in ascending order (stable compaction).
-__global__ void __launch_bounds__(1024) compact_masked_kernel(const uint8_t* __restrict__ is_masked,
-                                                              int L, int32_t* __restrict__ mrows,
-                                                              int32_t* __restrict__ mcount) {
+// Per sequence: the masked query rows in ascending order (stable compaction),
+// and the seed / newly-written flags packed 32 to a word.
+__global__ void __launch_bounds__(1024) prep_kernel(const uint8_t* __restrict__ is_masked,
+                                                    const uint8_t* __restrict__ is_seed,
+                                                    const uint8_t* __restrict__ is_new, int L,
+                                                    int32_t* __restrict__ mrows,
+                                                    int32_t* __restrict__ mcount,
+                                                    uint32_t* __restrict__ seedbits,
+                                                    uint32_t* __restrict__ newbits) {
   const int b = blockIdx.x;
+  const int W = (L + 31) / 32;
+  for (int i0 = threadIdx.x & ~31; i0 < W * 32; i0 += blockDim.x) {
+    const int i = i0 + (threadIdx.x & 31);
+    const bool fs = is_seed != nullptr && i < L && is_seed[(int64_t)b * L + i];
+    const bool fn = is_new != nullptr && i < L && is_new[(int64_t)b * L + i];
+    const uint32_t ws = __ballot_sync(0xffffffffu, fs), wn = __ballot_sync(0xffffffffu, fn);
+    if ((threadIdx.x & 31) == 0) {
+      if (seedbits) seedbits[(int64_t)b * W + i0 / 32] = ws;
+      if (newbits) newbits[(int64_t)b * W + i0 / 32] = wn;
+    }
+  }
+  if (mrows == nullptr) return;
   __shared__ int warp_sums[32];
   __shared__ int base;
   if (threadIdx.x == 0) base = 0;
@@ -66,18 +86,38 @@ __global__ void __launch_bounds__(1024) compact_masked_kernel(const uint8_t* __r
   if (threadIdx.x == 0) mcount[b] = base;
 }
 
-// d_x[b, j] = (accumulate ? d_x[b, j] : 0) + (1/Hq) sum_s part[b, s, j], s < nslices.
-__global__ void head_reduce_kernel(const float* __restrict__ part, int nslices, int L, float inv_hq,
-                                   int accumulate, int64_t total, float* __restrict__ dst) {
-  for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < total;
-       t += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t b = t / L;
-    const int j = (int)(t % L);
-    const float* p = part + b * nslices * L + j;
-    float s = 0.f;
-    for (int h = 0; h < nslices; ++h) s += p[(int64_t)h * L];
-    const float v = s * inv_hq;
-    dst[t] = accumulate ? dst[t] + v : v;
+// d_x[b, j] = (accumulate ? d_x[b, j] : 0) + (1/Hq) sum_s part[b, s, j], s < nslices,
+// for both statistics in one launch (part == nullptr skips one). Eight lanes per
+// position, each summing every eighth slice, then a shuffle reduction: one
+// round of memory latency whatever the head count.
+struct HeadReduce {
+  const float* part;
+  int nslices;
+  float* dst;
+};
+__global__ void __launch_bounds__(256) head_reduce_kernel(HeadReduce r0, HeadReduce r1, int B, int L,
+                                                          float inv_hq, int accumulate) {
+  const int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  const int64_t pos = t >> 3;
+  const int sub = (int)(t & 7);
+  if (pos >= (int64_t)B * L) return;  // whole groups of eight leave together
+  const unsigned mask = 0xFFu << (threadIdx.x & 24);
+  const int64_t b = pos / L;
+  const int j = (int)(pos % L);
+#pragma unroll
+  for (int which = 0; which < 2; ++which) {
+    const HeadReduce& r = which ? r1 : r0;
+    if (r.part == nullptr) continue;
+    const float* p = r.part + b * r.nslices * L + j;
+    float acc = 0.f;
+    for (int h = sub; h < r.nslices; h += 8) acc += p[(int64_t)h * L];
+    acc += __shfl_xor_sync(mask, acc, 4);
+    acc += __shfl_xor_sync(mask, acc, 2);
+    acc += __shfl_xor_sync(mask, acc, 1);
+    if (sub == 0) {
+      const float v = acc * inv_hq;
+      r.dst[pos] = accumulate ? r.dst[pos] + v : v;
+    }
   }
 }
 
@@ -343,10 +383,10 @@ cudaError_t launch_attention_tc(const AttnArgs& a, cudaStream_t stream, bool* ha
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t stream) {
   cudaError_t err;
   const bool need_din = a.d_in != nullptr && a.is_masked != nullptr;
-  if (need_din) {
-    compact_masked_kernel<<<a.B, 1024, 0, stream>>>(a.is_masked, a.L, a.mrows, a.mcount);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  }
+  prep_kernel<<<a.B, 1024, 0, stream>>>(a.is_masked, a.is_seed, a.is_new, a.L,
+                                        need_din ? a.mrows : nullptr, a.mcount, a.seedbits,
+                                        a.newbits);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
   bool handled = false;
   int din_slices = a.Hq;  // d_in partials: per query head (CUDA-core pass 2) or per kv head
   if (a.dtype == DD_BF16) {
@@ -362,25 +402,20 @@ cudaError_t launch_attention(const AttnArgs& a, cudaStream_t stream) {
     if (err != cudaSuccess) return err;
   }
   const int64_t total = (int64_t)a.B * a.L;
-  const int grid = (int)((total + 255) / 256 < 4096 ? (total + 255) / 256 : 4096);
+  HeadReduce rin{nullptr, 0, nullptr}, rout{nullptr, 0, nullptr};
   if (a.d_out) {
-    if (a.is_new) {
-      head_reduce_kernel<<<grid, 256, 0, stream>>>(a.dout_part, a.Hq, a.L, 1.f / a.Hq,
-                                                   a.accumulate, total, a.d_out);
-    } else if (!a.accumulate) {
-      cudaMemsetAsync(a.d_out, 0, total * sizeof(float), stream);
-    }
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    if (a.is_new) rout = HeadReduce{a.dout_part, a.Hq, a.d_out};
+    else if (!a.accumulate) cudaMemsetAsync(a.d_out, 0, total * sizeof(float), stream);
   }
   if (a.d_in) {
-    if (need_din) {
-      head_reduce_kernel<<<grid, 256, 0, stream>>>(a.din_part, din_slices, a.L, 1.f / a.Hq,
-                                                   a.accumulate, total, a.d_in);
-    } else if (!a.accumulate) {
-      cudaMemsetAsync(a.d_in, 0, total * sizeof(float), stream);
-    }
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    if (need_din) rin = HeadReduce{a.din_part, din_slices, a.d_in};
+    else if (!a.accumulate) cudaMemsetAsync(a.d_in, 0, total * sizeof(float), stream);
   }
+  if (rin.part || rout.part) {
+    head_reduce_kernel<<<(unsigned)((total * 8 + 255) / 256), 256, 0, stream>>>(
+        rin, rout, a.B, a.L, 1.f / a.Hq, a.accumulate);
+  }
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
   return cudaSuccess;
 }
 

@@ -45,7 +45,15 @@ struct P1Layout {
   static constexpr int kP = kV + kStages * kTile;
   static constexpr int kB2 = kP + 2 * kAtom;          // P: 128 rows x 128 columns bf16
   static constexpr int kB2Bytes = 2 * 16 * 128;       // 16 rows x 128 columns bf16
-  static constexpr int kBar = kB2 + kStages * kB2Bytes;
+  // staging for up to kStaged seed rows of the step t-1 cache per stage (K then V rows)
+  static constexpr int kStaged = 16;
+  static constexpr int kRowBytes = D * 2;
+  static constexpr int kStage = kB2 + kStages * kB2Bytes;
+  static constexpr int kStageBytes = 2 * kStaged * kRowBytes;
+  // packed seed / newly-written flags of the whole sequence
+  static constexpr int kMask = kStage + kStages * kStageBytes;
+  static constexpr int kMaskWords = kTcMaxL / 32;
+  static constexpr int kBar = kMask + 2 * kMaskWords * 4;
   static constexpr int kBytes = kBar + 256;
   // TMEM columns
   static constexpr uint32_t kS0 = 0, kS1 = 128, kO = 256, kSt = 256 + D;
@@ -67,6 +75,7 @@ struct P1Bars {
 struct P1Params {
   const __nv_bfloat16 *q, *k_cur, *v_cur, *k_prev, *v_prev;
   const uint8_t *is_seed, *is_new;
+  const uint32_t *seedbits, *newbits;  // [B, ceil(L/32)]
   int L, Hq, Hkv;
   float scale_log2;
   __nv_bfloat16* out;
@@ -82,7 +91,8 @@ __device__ __forceinline__ uint4 ldg16(const void* p) {
 template <int D>
 __global__ void __launch_bounds__(kP1Threads, 1)
 attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-               const __grid_constant__ CUtensorMap tmV, const P1Params p) {
+               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKp,
+               const __grid_constant__ CUtensorMap tmVp, const P1Params p) {
   using Lay = P1Layout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -142,10 +152,27 @@ attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       for (int ac = 0; ac < D / 64; ++ac)
         tma_load_4d(smem + Lay::kQ + ac * kAtom, &tmQ, ac * 64, h, q0, b, &bars->q_full);
     }
+    // the sequence's packed flags into shared memory
+    uint32_t* seedw = reinterpret_cast<uint32_t*>(smem + Lay::kMask);
+    uint32_t* neww = seedw + Lay::kMaskWords;
+    const int W = (L + 31) / 32;
+    for (int w = lane; w < W; w += 32) {
+      seedw[w] = p.seedbits[(int64_t)b * W + w];
+      neww[w] = p.newbits[(int64_t)b * W + w];
+    }
+    __syncwarp();
+    // Tile j: K/V from the current input, plus (same barrier) up to kStaged
+    // seed rows of the step t-1 cache into the stage's staging area.
     auto issue = [&](int j) {
       const int s = j % kStages;
       if (lane == 0) {
-        mbar_expect_tx(&bars->kv_full[s], kTxKV);
+        int n = 0;
+        for (int w = 0; w < 4; ++w) {
+          const int wi = j * 4 + w;
+          n += wi < W ? __popc(seedw[wi]) : 0;
+        }
+        n = min(n, Lay::kStaged);
+        mbar_expect_tx(&bars->kv_full[s], kTxKV + 2u * n * Lay::kRowBytes);
 #pragma unroll
         for (int ac = 0; ac < D / 64; ++ac) {
           tma_load_4d(smem + Lay::kK + s * Lay::kTile + ac * kAtom, &tmK, ac * 64, g, j * kBN, b,
@@ -153,43 +180,66 @@ attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           tma_load_4d(smem + Lay::kV + s * Lay::kTile + ac * kAtom, &tmV, ac * 64, g, j * kBN, b,
                       &bars->kv_full[s]);
         }
+        uint8_t* stg = smem + Lay::kStage + s * Lay::kStageBytes;
+        int slot = 0;
+        for (int w = 0; w < 4 && slot < n; ++w) {
+          const int wi = j * 4 + w;
+          uint32_t bits = wi < W ? seedw[wi] : 0u;
+          while (bits && slot < n) {
+            const int r = w * 32 + __ffs(bits) - 1;
+            bits &= bits - 1;
+            tma_load_4d(stg + slot * Lay::kRowBytes, &tmKp, 0, g, j * kBN + r, b,
+                        &bars->kv_full[s]);
+            tma_load_4d(stg + (Lay::kStaged + slot) * Lay::kRowBytes, &tmVp, 0, g, j * kBN + r,
+                        b, &bars->kv_full[s]);
+            ++slot;
+          }
+        }
       }
     };
     auto finalize = [&](int j) -> bool {
       const int s = j % kStages;
       if (!wait_bounded(&bars->kv_full[s], (j / kStages) & 1, p.spin, abort_flag)) return false;
       const int col0 = j * kBN;
+      const uint32_t stg = sbase + Lay::kStage + s * Lay::kStageBytes;
+      const bool is_v = lane >= 16;
+      const int ch = lane & 15;
       // drafting view: seed columns read the step t-1 cache
-#pragma unroll
+      int slot = 0;
       for (int w = 0; w < 4; ++w) {
-        const int c = col0 + w * 32 + lane;
-        const bool f = p.is_seed != nullptr && c < L && p.is_seed[(int64_t)b * L + c] != 0;
-        uint32_t bits = __ballot_sync(0xffffffffu, f);
+        const int wi = j * 4 + w;
+        uint32_t bits = wi < W ? seedw[wi] : 0u;
         while (bits) {
           const int r = w * 32 + __ffs(bits) - 1;
           bits &= bits - 1;
-          const int64_t off = (((int64_t)b * L + col0 + r) * p.Hkv + g) * D;
-          const bool is_v = lane >= 16;
-          const int ch = lane & 15;
           if (ch < D / 8) {
-            const __nv_bfloat16* src = (is_v ? p.v_prev : p.k_prev) + off + ch * 8;
-            const uint4 val = ldg16(src);
+            uint4 val;
+            if (slot < Lay::kStaged) {
+              const uint32_t src =
+                  stg + ((is_v ? Lay::kStaged : 0) + slot) * Lay::kRowBytes + ch * 16;
+              asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                           : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
+                           : "r"(src));
+            } else {
+              val = ldg16((is_v ? p.v_prev : p.k_prev) +
+                          (((int64_t)b * L + col0 + r) * p.Hkv + g) * D + ch * 8);
+            }
             const uint32_t dst = sbase + (is_v ? Lay::kV : Lay::kK) + s * Lay::kTile +
                                  (ch / 8) * kAtom + sw128(r, ch & 7);
             st_shared_v4(dst, val.x, val.y, val.z, val.w);
           }
+          ++slot;
         }
       }
       // row 1 of the statistics operand: the tile's newly-written flags
       if (lane < 16) {
+        const int wi = j * 4 + lane / 4;
+        const uint32_t byte = ((wi < W ? neww[wi] : 0u) >> ((lane & 3) * 8)) & 0xFFu;
         uint32_t w4[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int c0 = col0 + lane * 8 + 2 * e;
-          const bool n0 = p.is_new != nullptr && c0 < L && p.is_new[(int64_t)b * L + c0];
-          const bool n1 = p.is_new != nullptr && c0 + 1 < L && p.is_new[(int64_t)b * L + c0 + 1];
-          w4[e] = (n0 ? 0x3F80u : 0u) | (n1 ? 0x3F800000u : 0u);
-        }
+        for (int e = 0; e < 4; ++e)
+          w4[e] = ((byte >> (2 * e)) & 1u ? 0x3F80u : 0u) |
+                  ((byte >> (2 * e + 1)) & 1u ? 0x3F800000u : 0u);
         st_shared_v4(sbase + Lay::kB2 + s * Lay::kB2Bytes + (lane / 8) * 2048 + sw128(1, lane & 7),
                      w4[0], w4[1], w4[2], w4[3]);
       }
@@ -344,8 +394,8 @@ attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         uint32_t w[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float a = live ? exp2f(fmaf(s[cc * 8 + 2 * e], c2, -m)) : 0.f;
-          const float bb = live ? exp2f(fmaf(s[cc * 8 + 2 * e + 1], c2, -m)) : 0.f;
+          const float a = live ? fast_exp2(fmaf(s[cc * 8 + 2 * e], c2, -m)) : 0.f;
+          const float bb = live ? fast_exp2(fmaf(s[cc * 8 + 2 * e + 1], c2, -m)) : 0.f;
           w[e] = pack_bf16(a, bb);
         }
         st_shared_v4(sP + (cc / 8) * kAtom + sw128(r, cc & 7), w[0], w[1], w[2], w[3]);
@@ -465,7 +515,7 @@ struct P2Bars {
 
 struct P2Params {
   const __nv_bfloat16 *q, *k_prev;
-  const uint8_t* is_seed;
+  const uint32_t* seedbits;
   const float* lse;
   const int32_t *mrows, *mcount;
   int L, Hq, Hkv;
@@ -525,12 +575,13 @@ attn_p2_kernel(const __grid_constant__ CUtensorMap tmK, const P2Params p) {
         for (int ac = 0; ac < D / 64; ++ac)
           tma_load_4d(smem + Lay::kK + ac * kAtom, &tmK, ac * 64, g, col0, b, &bars->k_full);
       }
+      const int W = (L + 31) / 32;
+      uint32_t seedword = 0;
+      if (lane < 4 && kt * 4 + lane < W) seedword = p.seedbits[(int64_t)b * W + kt * 4 + lane];
       if (wait_bounded(&bars->k_full, 0, p.spin, abort_flag)) {
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
-          const int c = col0 + w * 32 + lane;
-          const bool f = p.is_seed != nullptr && c < L && p.is_seed[(int64_t)b * L + c] != 0;
-          uint32_t bits = __ballot_sync(0xffffffffu, f);
+          uint32_t bits = __shfl_sync(0xffffffffu, seedword, w);
           while (bits) {
             const int r = w * 32 + __ffs(bits) - 1;
             bits &= bits - 1;
@@ -623,10 +674,10 @@ attn_p2_kernel(const __grid_constant__ CUtensorMap tmK, const P2Params p) {
 #pragma unroll
       for (int c4 = 0; c4 < kBN / 4; ++c4) {
         const float4 l4 = lv[c4];
-        a0 += exp2f(fmaf(s[4 * c4 + 0], c2, -l4.x));
-        a1 += exp2f(fmaf(s[4 * c4 + 1], c2, -l4.y));
-        a0 += exp2f(fmaf(s[4 * c4 + 2], c2, -l4.z));
-        a1 += exp2f(fmaf(s[4 * c4 + 3], c2, -l4.w));
+        a0 += fast_exp2(fmaf(s[4 * c4 + 0], c2, -l4.x));
+        a1 += fast_exp2(fmaf(s[4 * c4 + 1], c2, -l4.y));
+        a0 += fast_exp2(fmaf(s[4 * c4 + 2], c2, -l4.z));
+        a1 += fast_exp2(fmaf(s[4 * c4 + 3], c2, -l4.w));
       }
       acc += a0 + a1;
       fence_before_sync();
@@ -671,11 +722,28 @@ bool make_map(CUtensorMap* map, const void* base, int D, int H, int L, int B) {
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Rows of the step t-1 cache: box = one whole head row (D elements), no swizzle.
+bool make_row_map(CUtensorMap* map, const void* base, int D, int H, int L, int B) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)L, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)L * H * D * 2};
+  cuuint32_t box[4] = {(cuuint32_t)D, 1, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int D>
 cudaError_t launch_p1(const AttnArgs& a, cudaStream_t stream) {
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, tkp, tvp;
+  // without seeds the cache maps are never read; point them at the current K/V
+  const void* kp = a.is_seed ? a.k_prev : a.k_cur;
+  const void* vp = a.is_seed ? a.v_prev : a.v_cur;
   if (!make_map(&tq, a.q, D, a.Hq, a.L, a.B) || !make_map(&tk, a.k_cur, D, a.Hkv, a.L, a.B) ||
-      !make_map(&tv, a.v_cur, D, a.Hkv, a.L, a.B))
+      !make_map(&tv, a.v_cur, D, a.Hkv, a.L, a.B) ||
+      !make_row_map(&tkp, kp, D, a.Hkv, a.L, a.B) || !make_row_map(&tvp, vp, D, a.Hkv, a.L, a.B))
     return cudaErrorInvalidValue;
   const int smem = P1Layout<D>::kBytes + 1024;
   static int configured[64] = {};
@@ -694,6 +762,8 @@ cudaError_t launch_p1(const AttnArgs& a, cudaStream_t stream) {
   p.v_prev = static_cast<const __nv_bfloat16*>(a.v_prev);
   p.is_seed = a.is_seed;
   p.is_new = a.is_new;
+  p.seedbits = a.seedbits;
+  p.newbits = a.newbits;
   p.L = a.L;
   p.Hq = a.Hq;
   p.Hkv = a.Hkv;
@@ -703,7 +773,7 @@ cudaError_t launch_p1(const AttnArgs& a, cudaStream_t stream) {
   p.dout_part = a.dout_part;
   p.spin = spin_limit();
   dim3 grid((a.L + kBM - 1) / kBM, a.Hq, a.B);
-  attn_p1_kernel<D><<<grid, kP1Threads, smem, stream>>>(tq, tk, tv, p);
+  attn_p1_kernel<D><<<grid, kP1Threads, smem, stream>>>(tq, tk, tv, tkp, tvp, p);
   return cudaGetLastError();
 }
 
@@ -723,7 +793,7 @@ cudaError_t launch_p2(const AttnArgs& a, cudaStream_t stream) {
   P2Params p;
   p.q = static_cast<const __nv_bfloat16*>(a.q);
   p.k_prev = static_cast<const __nv_bfloat16*>(a.k_prev);
-  p.is_seed = a.is_seed;
+  p.seedbits = a.seedbits;
   p.lse = a.lse;
   p.mrows = a.mrows;
   p.mcount = a.mcount;

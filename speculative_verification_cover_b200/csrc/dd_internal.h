@@ -36,11 +36,13 @@ struct AttnArgs {
   float* din_part;      // [B, Hq, L]
   int32_t* mrows;       // [B, L] masked rows of each sequence, ascending
   int32_t* mcount;      // [B]
+  uint32_t* seedbits;   // [B, ceil(L/32)] packed is_seed
+  uint32_t* newbits;    // [B, ceil(L/32)] packed is_new
 };
 
 // Workspace layout shared by the entry point and the kernels.
 struct AttnWorkspace {
-  size_t dout_off, din_off, mrows_off, mcount_off, total;
+  size_t dout_off, din_off, mrows_off, mcount_off, seedbits_off, newbits_off, total;
 };
 AttnWorkspace attn_workspace_layout(int B, int L, int Hq);
 
@@ -49,7 +51,8 @@ cudaError_t launch_attention(const AttnArgs& a, cudaStream_t stream);
 cudaError_t launch_verify_logits(const void* lt, const void* lm, dd_dtype dtype, int B, int R,
                                  int V, int64_t ld, int pos_offset, float temperature,
                                  uint64_t seed, uint64_t step, const dd_row_stats& out,
-                                 cudaStream_t stream);
+                                 void* workspace, cudaStream_t stream);
+size_t verify_workspace_bytes(int B, int R, int V, dd_dtype dtype);
 
 cudaError_t launch_coupled_gumbel(uint64_t seed, uint64_t step, int B, int R, int V, int64_t ld,
                                   int pos_offset, float* g, cudaStream_t stream);
@@ -69,6 +72,8 @@ cudaError_t launch_selftest_wait(uint32_t limit, cudaStream_t stream);
 
 // Largest L dd_select_seeds handles (keys of one sequence live in shared memory).
 constexpr int kSelectMaxL = 24576;
+// Longest sequence the tensor-core attention handles (packed masks live in shared memory).
+constexpr int kTcMaxL = 32768;
 constexpr int kSelectMaxK = 1024;
 
 }  // namespace dd

@@ -7,7 +7,7 @@ namespace dd {
 
 namespace {
 
-constexpr int kSelThreads = 1024;
+constexpr int kSelThreads = 512;
 
 // Order-preserving map of a float onto uint32 (larger float -> larger key).
 __device__ __forceinline__ uint32_t orderable(float f) {
@@ -15,95 +15,139 @@ __device__ __forceinline__ uint32_t orderable(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// Block-wide exclusive prefix sum of one int per thread (blockDim.x multiple of 32).
+__device__ __forceinline__ int block_exclusive_sum(int x, int* warp_tmp, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int incl = x;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) warp_tmp[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int v = lane < nw ? warp_tmp[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += t;
+    }
+    if (lane < nw) warp_tmp[lane] = v;  // inclusive over warps
+    if (lane == nw - 1) *total = v;
+  }
+  __syncthreads();
+  const int before = warp > 0 ? warp_tmp[warp - 1] : 0;
+  const int r = before + incl - x;
+  __syncthreads();
+  return r;
+}
+
 // One CTA per sequence.
 //   score_i = u_i (1 + d_in_i) / (1 + d_out_i) on eligible positions with a row.
-// Candidates get the 64-bit key (orderable(score) << 32) | (0xFFFFFFFF - i):
-// keys are distinct, larger key = higher score, then lower position. The k-th
-// largest key is found by an MSB-first radix select (8 passes of 8 bits) over
-// keys in shared memory; the chosen positions are ranked by counting.
+// The k-th largest score (as an order-preserving 32-bit key) is found by an
+// MSB-first radix select, 8 bits per pass; positions tied with it are taken in
+// ascending order up to k (a block prefix count); the chosen positions are
+// ranked by (score descending, position ascending).
 __global__ void __launch_bounds__(kSelThreads)
 select_seeds_kernel(const float* __restrict__ entropy, int R, int pos_offset,
                     const float* __restrict__ d_in, const float* __restrict__ d_out,
                     const uint8_t* __restrict__ eligible, int L, int k,
                     int32_t* __restrict__ seeds, uint8_t* __restrict__ is_seed,
                     float* __restrict__ score) {
-  extern __shared__ unsigned long long keys[];  // [L]; 0 = not a candidate
+  extern __shared__ uint32_t skey[];  // [L] orderable score; 0 = not a candidate
   __shared__ unsigned int hist[256];
-  __shared__ unsigned int warp_tot[kSelThreads / 32];
-  __shared__ unsigned long long prefix_s;
-  __shared__ int need_s, ncand_s, nsel_s;
+  __shared__ int warp_tmp[32];
+  __shared__ int total_s, nsel_s, ncand_s;
+  __shared__ uint32_t prefix_s;
+  __shared__ int need_s;
   __shared__ unsigned long long chosen[kSelectMaxK];
-
   const int b = blockIdx.x;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
   if (threadIdx.x == 0) { ncand_s = 0; nsel_s = 0; }
+  for (int t = threadIdx.x; t < 256; t += blockDim.x) hist[t] = 0u;
   __syncthreads();
   int my_cand = 0;
   for (int i = threadIdx.x; i < L; i += blockDim.x) {
     const int64_t bi = (int64_t)b * L + i;
     const int r = i - pos_offset;
     float s = -INFINITY;
-    unsigned long long key = 0ull;
+    uint32_t key = 0u;
     if (eligible[bi] && r >= 0 && r < R) {
       const float u = entropy[(int64_t)b * R + r];
       s = u * (1.f + d_in[bi]) / (1.f + d_out[bi]);
-      key = ((unsigned long long)orderable(s) << 32) | (0xFFFFFFFFu - (uint32_t)i);
+      key = orderable(s);
       ++my_cand;
     }
-    keys[i] = key;
+    skey[i] = key;
     if (score) score[bi] = s;
   }
-  atomicAdd(&ncand_s, my_cand);
+  if (my_cand) atomicAdd(&ncand_s, my_cand);
   __syncthreads();
   const int ncand = ncand_s;
   const int kk = k < ncand ? k : ncand;
-  unsigned long long thresh = 1ull;  // select keys >= thresh (all candidates by default)
+  // ---- the kk-th largest key (keys are > 0 for candidates)
+  uint32_t thresh = 1u;
+  int need = 0;  // how many keys equal to thresh are taken
   if (kk > 0 && kk < ncand) {
-    unsigned long long prefix = 0ull;
-    int need = kk;  // how many keys >= the final threshold remain to be found below prefix
-    for (int shift = 56; shift >= 0; shift -= 8) {
-      for (int t = threadIdx.x; t < 256; t += blockDim.x) hist[t] = 0u;
-      __syncthreads();
-      const unsigned long long hmask = shift == 56 ? 0ull : (~0ull << (shift + 8));
+    uint32_t prefix = 0u;
+    int want = kk;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      const uint32_t hmask = shift == 24 ? 0u : (0xFFFFFFFFu << (shift + 8));
       for (int i = threadIdx.x; i < L; i += blockDim.x) {
-        const unsigned long long key = keys[i];
-        if (key != 0ull && (key & hmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+        const uint32_t key = skey[i];
+        if (key != 0u && (key & hmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
       }
       __syncthreads();
-      // thread t < 256 takes digit 255 - t; inclusive scan gives #keys with digit >= 255 - t
-      unsigned int c = 0u, incl = 0u;
-      if (threadIdx.x < 256) {
-        c = hist[255 - threadIdx.x];
-        incl = c;
+      if (threadIdx.x < 32) {
+        // lane handles digits 255-8*lane .. 248-8*lane (descending)
+        unsigned int c[8], sum = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) { c[e] = hist[255 - 8 * lane - e]; sum += c[e]; }
+        unsigned int incl = sum;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-          const unsigned int t2 = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += t2;
+          const unsigned int t = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += t;
         }
-        if (lane == 31) warp_tot[warp] = incl;
-      }
-      __syncthreads();
-      if (threadIdx.x < 256) {
-        for (int w = 0; w < warp; ++w) incl += warp_tot[w];
-        if (incl >= (unsigned)need && incl - c < (unsigned)need) {
-          const unsigned long long digit = 255 - threadIdx.x;
-          prefix_s = prefix | (digit << shift);
-          need_s = need - (int)(incl - c);
+        unsigned int run = incl - sum;  // keys with a larger digit than this lane's first
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          if (run < (unsigned)want && run + c[e] >= (unsigned)want) {
+            prefix_s = prefix | ((uint32_t)(255 - 8 * lane - e) << shift);
+            need_s = want - (int)run;
+          }
+          run += c[e];
         }
       }
       __syncthreads();
       prefix = prefix_s;
-      need = need_s;
+      want = need_s;
+      for (int t = threadIdx.x; t < 256; t += blockDim.x) hist[t] = 0u;
       __syncthreads();
     }
-    thresh = prefix;  // the kk-th largest key itself
+    thresh = prefix;
+    need = want;
   }
-  // collect the chosen keys
-  for (int i = threadIdx.x; i < L; i += blockDim.x) {
-    const unsigned long long key = keys[i];
-    const bool sel = kk > 0 && key != 0ull && key >= thresh;
-    if (sel) chosen[atomicAdd(&nsel_s, 1)] = key;
-    if (is_seed) is_seed[(int64_t)b * L + i] = sel ? 1 : 0;
+  // ---- choose: keys above the threshold, then the first `need` ties by position
+  for (int i0 = 0; i0 < L; i0 += blockDim.x) {
+    const int i = i0 + threadIdx.x;
+    const uint32_t key = i < L ? skey[i] : 0u;
+    const bool tie = kk > 0 && key != 0u && key == thresh && kk < ncand;
+    const int before = block_exclusive_sum(tie ? 1 : 0, warp_tmp, &total_s);
+    if (i < L) {
+      const bool sel = kk > 0 && key != 0u && (kk >= ncand ? true : (key > thresh ||
+                                                                     (tie && before < need)));
+      if (sel) {
+        const int slot = atomicAdd(&nsel_s, 1);
+        chosen[slot] = ((unsigned long long)key << 32) | (0xFFFFFFFFu - (uint32_t)i);
+      }
+      if (is_seed) is_seed[(int64_t)b * L + i] = sel ? 1 : 0;
+    }
+    if (kk < ncand) {
+      need -= total_s;
+      if (need < 0) need = 0;
+    }
   }
   __syncthreads();
   const int nsel = nsel_s;
@@ -117,7 +161,7 @@ select_seeds_kernel(const float* __restrict__ entropy, int R, int pos_offset,
 }
 
 // One CTA per sequence; accepted[b] = all decided positions KEEP.
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(1024)
 decide_kernel(dd_decide_params p, const int32_t* __restrict__ tokens,
               const uint8_t* __restrict__ is_seed, const uint8_t* __restrict__ eligible,
               dd_row_stats st, int L, int R, int pos_offset, uint8_t* __restrict__ decision,
@@ -189,13 +233,13 @@ cudaError_t launch_select_seeds(const float* entropy, int R, int pos_offset, con
                                 const float* d_out, const uint8_t* eligible, int B, int L, int k,
                                 int32_t* seeds, uint8_t* is_seed, float* score,
                                 cudaStream_t stream) {
-  const size_t smem = (size_t)L * sizeof(unsigned long long);
+  const size_t smem = (size_t)L * sizeof(uint32_t);
   static thread_local int configured_for = -1;
   const DeviceInfo& dev = device_info();
   if (configured_for != dev.device) {
     cudaError_t e = cudaFuncSetAttribute(select_seeds_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)(kSelectMaxL * sizeof(unsigned long long)));
+                                         (int)(kSelectMaxL * sizeof(uint32_t)));
     if (e != cudaSuccess) return e;
     configured_for = dev.device;
   }
@@ -209,7 +253,7 @@ cudaError_t launch_decide(const dd_decide_params& p, const int32_t* tokens,
                           const dd_row_stats& stats, int B, int L, int R, int pos_offset,
                           uint8_t* decision, int32_t* new_tokens, uint8_t* accepted,
                           cudaStream_t stream) {
-  decide_kernel<<<B, 256, 0, stream>>>(p, tokens, is_seed, eligible, stats, L, R, pos_offset,
+  decide_kernel<<<B, 1024, 0, stream>>>(p, tokens, is_seed, eligible, stats, L, R, pos_offset,
                                        decision, new_tokens, accepted);
   return cudaGetLastError();
 }

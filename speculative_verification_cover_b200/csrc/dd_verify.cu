@@ -4,30 +4,35 @@
 // One streaming read of the verifier logits l and the drafter logits m of each
 // verified row produces: LSE of both, argmax of both, the verifier's max
 // probability, its entropy (the uncertainty u of COVER's seed score),
-// KL(drafter || verifier), and at T > 0 the coupled Gumbel-max samples of
-// both with the same Philox noise.
+// KL(drafter || verifier), and at T > 0 the coupled Gumbel-max samples of both
+// with the same Philox noise.
 //
-// Work decomposition: a row is split into C contiguous segments, one CTA each;
-// the C CTAs of a row form a thread-block cluster and merge their partial
-// states through distributed shared memory, so no global scratch is needed.
-// Each thread streams 16-byte vectors with no-L1-allocate loads, four vectors
-// of each matrix in flight, and keeps an online (running-max rescaled) state:
-//   s1 = sum e^{x - M},  s2 = sum e^{x - M} (x - M) log2(e),  sk = sum e^{m - Md}(m - l)
-// from which LSE = M + ln s1, H = ln s1 - s2 ln2 / s1, conf = 1 / s1,
-// KL = sk_d / s1_d + (M_t - M_d) + ln(s1_t / s1_d).
-#include <cooperative_groups.h>
-
+// Work decomposition: the 16-byte vectors of all rows form one index space
+// (rows x vectors per row); it is split into equal contiguous ranges, one per
+// persistent CTA (several per SM), so every SM streams the same number of bytes
+// whatever B, R and V are. A CTA's range is one to a few row pieces; in each
+// piece its 256 threads stride over the vectors four at a time with streaming
+// 16-byte loads, folding each into an online (running-max rescaled) state kept
+// in float2 lanes so pairs of entries use the packed fp32 pipe:
+//   s1 = sum e^{x - M},  s2 = sum e^{x - M} (x - M) log2(e),  sk = sum e^{m - Md}(m - l).
+// At the end of a piece the CTA reduces its state to one partial per
+// (row, CTA) in the workspace; a small second kernel merges a row's partials:
+//   LSE = M + ln s1, H = ln s1 - s2 ln2 / s1, conf = 1 / s1,
+//   KL = sk_d / s1_d + (M_t - M_d) + ln(s1_t / s1_d).
 #include "dd_common.cuh"
 #include "dd_internal.h"
-
-namespace cg = cooperative_groups;
+#include "dd_tc.cuh"
 
 namespace dd {
 
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kUnroll = 4;
+constexpr int kVThreads = 256;
+template <bool SAMPLE>
+struct VCfg {
+  static constexpr int kMinBlocks = SAMPLE ? 2 : 3;  // resident CTAs per SM
+};
+constexpr int kMaxGridPerSm = 3;
 
 struct Partial {
   float mt, s1t, s2t;  // verifier: max, sum e, sum e*y (log2 units)
@@ -36,6 +41,12 @@ struct Partial {
   float bt, lt_at;     // best coupled score of l, and l at that index
   float bd;            // best coupled score of m
   int it, id;          // their indices
+  int pad[3];
+};
+static_assert(sizeof(Partial) == 64, "partial record is 64 bytes");
+
+struct NoiseKey {
+  uint32_t k0, k1, step;
 };
 
 __device__ __forceinline__ void init(Partial& p) {
@@ -47,96 +58,257 @@ __device__ __forceinline__ void init(Partial& p) {
   p.it = p.id = 0x7fffffff;
 }
 
-// Accumulate N consecutive vocabulary entries starting at index v0.
-template <int N, bool SAMPLE>
-__device__ __forceinline__ void accumulate(Partial& p, const float (&l)[N], const float (&m)[N],
-                                           const float (&g)[N], int v0, float invT) {
-  // --- verifier: maximum, argmax (lowest index), online rescale
-  float cm = l[0];
+// Per-thread accumulator: the sums are float2 so that pairs of vocabulary
+// entries go through the packed fp32 pipe (FFMA2 / FADD2) and each sum has two
+// independent dependency chains.
+struct Acc {
+  float mt, md;
+  float2 s1t, s2t, s1d, skd;
+  int at, ad;
+  float bt, lt_at, bd;
+  int it, id;
+};
+
+__device__ __forceinline__ void init(Acc& a) {
+  a.mt = a.md = -INFINITY;
+  a.s1t = a.s2t = a.s1d = a.skd = make_float2(0.f, 0.f);
+  a.at = a.ad = 0x7fffffff;
+  a.bt = a.bd = -INFINITY;
+  a.lt_at = 0.f;
+  a.it = a.id = 0x7fffffff;
+}
+
+__device__ __forceinline__ Partial to_partial(const Acc& a) {
+  Partial p;
+  p.mt = a.mt;
+  p.s1t = a.s1t.x + a.s1t.y;
+  p.s2t = a.s2t.x + a.s2t.y;
+  p.md = a.md;
+  p.s1d = a.s1d.x + a.s1d.y;
+  p.skd = a.skd.x + a.skd.y;
+  p.at = a.at;
+  p.ad = a.ad;
+  p.bt = a.bt;
+  p.lt_at = a.lt_at;
+  p.bd = a.bd;
+  p.it = a.it;
+  p.id = a.id;
+  return p;
+}
+
+__device__ __forceinline__ float2 ex2x2(float2 y) {
+  return make_float2(fast_exp2(y.x), fast_exp2(y.y));
+}
+
+__device__ __forceinline__ uint32_t hmax2_bits(uint32_t a, uint32_t b) {
+  __nv_bfloat162 x = *reinterpret_cast<__nv_bfloat162*>(&a);
+  __nv_bfloat162 y = *reinterpret_cast<__nv_bfloat162*>(&b);
+  __nv_bfloat162 r = __hmax2(x, y);
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+
+// Fold NV 16-byte vectors of each matrix (vector k starts at vocabulary index v0[k],
+// indices increasing with k). l/m: the unpacked values; lw/mw: the raw words.
+template <typename T, bool SAMPLE, int NV>
+__device__ __forceinline__ void fold(Acc& a, const uint4 (&lw)[NV], const uint4 (&mw)[NV],
+                                     const int (&v0)[NV], int pos, int b, const NoiseKey& key,
+                                     float invT);
+
+template <typename T>
+struct Unpack;
+template <>
+struct Unpack<__nv_bfloat16> {
+  static constexpr int N = 8;
+  __device__ static void run(const uint4& u, float2 (&x)[4]) {
+    x[0] = make_float2(bf16lo(u.x), bf16hi(u.x));
+    x[1] = make_float2(bf16lo(u.y), bf16hi(u.y));
+    x[2] = make_float2(bf16lo(u.z), bf16hi(u.z));
+    x[3] = make_float2(bf16lo(u.w), bf16hi(u.w));
+  }
+  __device__ static float vmax(const uint4& u) {
+    const uint32_t h = hmax2_bits(hmax2_bits(u.x, u.y), hmax2_bits(u.z, u.w));
+    return fmaxf(bf16lo(h), bf16hi(h));
+  }
+};
+template <>
+struct Unpack<float> {
+  static constexpr int N = 4;
+  __device__ static void run(const uint4& u, float2 (&x)[2]) {
+    x[0] = make_float2(__uint_as_float(u.x), __uint_as_float(u.y));
+    x[1] = make_float2(__uint_as_float(u.z), __uint_as_float(u.w));
+  }
+  __device__ static float vmax(const uint4& u) {
+    return fmaxf(fmaxf(__uint_as_float(u.x), __uint_as_float(u.y)),
+                 fmaxf(__uint_as_float(u.z), __uint_as_float(u.w)));
+  }
+};
+
+template <typename T, bool SAMPLE, int NV>
+__device__ __forceinline__ void fold(Acc& a, const uint4 (&lw)[NV], const uint4 (&mw)[NV],
+                                     const int (&v0)[NV], int pos, int b, const NoiseKey& key,
+                                     float invT) {
+  constexpr int VEC = Unpack<T>::N, NP = VEC / 2;
+  float2 L[NV][NP], M[NV][NP];
 #pragma unroll
-  for (int i = 1; i < N; ++i) cm = fmaxf(cm, l[i]);
-  if (cm > p.mt) {
-    int a = v0 + N - 1;
+  for (int k = 0; k < NV; ++k) {
+    Unpack<T>::run(lw[k], L[k]);
+    Unpack<T>::run(mw[k], M[k]);
+  }
+  // --- maxima; a new maximum (rare after the first few vectors) rescales the sums
+  float cm = Unpack<T>::vmax(lw[0]), dm = Unpack<T>::vmax(mw[0]);
 #pragma unroll
-    for (int i = N - 1; i >= 0; --i)
-      if (l[i] == cm) a = v0 + i;
-    if (p.mt != -INFINITY) {
-      const float dl = (p.mt - cm) * kLog2e;
+  for (int k = 1; k < NV; ++k) {
+    cm = fmaxf(cm, Unpack<T>::vmax(lw[k]));
+    dm = fmaxf(dm, Unpack<T>::vmax(mw[k]));
+  }
+  // A new maximum is rare after the first vectors of a row: branch on a warp
+  // vote so the rescale / argmax scan is skipped, not executed predicated.
+  if (__any_sync(__activemask(), cm > a.mt) && cm > a.mt) {
+    int idx = 0x7fffffff;
+#pragma unroll
+    for (int k = NV - 1; k >= 0; --k)
+#pragma unroll
+      for (int e = NP - 1; e >= 0; --e) {
+        if (L[k][e].y == cm) idx = v0[k] + 2 * e + 1;
+        if (L[k][e].x == cm) idx = v0[k] + 2 * e;
+      }
+    if (a.mt != -INFINITY) {
+      const float dl = (a.mt - cm) * kLog2e;
       const float f = exp2f(dl);
-      p.s2t = f * (p.s2t + dl * p.s1t);
-      p.s1t = f * p.s1t;
+      const float2 f2 = make_float2(f, f), dl2 = make_float2(dl, dl);
+      a.s2t = __fmul2_rn(f2, __ffma2_rn(dl2, a.s1t, a.s2t));
+      a.s1t = __fmul2_rn(f2, a.s1t);
     }
-    p.mt = cm;
-    p.at = a;
+    a.mt = cm;
+    a.at = idx;
   }
-  const float mt2 = p.mt * kLog2e;
+  if (__any_sync(__activemask(), dm > a.md) && dm > a.md) {
+    int idx = 0x7fffffff;
 #pragma unroll
-  for (int i = 0; i < N; ++i) {
-    const float y = fmaf(l[i], kLog2e, -mt2);
-    const float e = fast_exp2(y);
-    p.s1t += e;
-    p.s2t = fmaf(e, y, p.s2t);
-  }
-  // --- drafter
-  float dm = m[0];
+    for (int k = NV - 1; k >= 0; --k)
 #pragma unroll
-  for (int i = 1; i < N; ++i) dm = fmaxf(dm, m[i]);
-  if (dm > p.md) {
-    int a = v0 + N - 1;
-#pragma unroll
-    for (int i = N - 1; i >= 0; --i)
-      if (m[i] == dm) a = v0 + i;
-    if (p.md != -INFINITY) {
-      const float f = exp2f((p.md - dm) * kLog2e);
-      p.s1d *= f;
-      p.skd *= f;
+      for (int e = NP - 1; e >= 0; --e) {
+        if (M[k][e].y == dm) idx = v0[k] + 2 * e + 1;
+        if (M[k][e].x == dm) idx = v0[k] + 2 * e;
+      }
+    if (a.md != -INFINITY) {
+      const float f = exp2f((a.md - dm) * kLog2e);
+      const float2 f2 = make_float2(f, f);
+      a.s1d = __fmul2_rn(f2, a.s1d);
+      a.skd = __fmul2_rn(f2, a.skd);
     }
-    p.md = dm;
-    p.ad = a;
+    a.md = dm;
+    a.ad = idx;
   }
-  const float md2 = p.md * kLog2e;
+  const float2 l2e = make_float2(kLog2e, kLog2e);
+  const float2 nmt = make_float2(-a.mt * kLog2e, -a.mt * kLog2e);
+  const float2 nmd = make_float2(-a.md * kLog2e, -a.md * kLog2e);
+  const float2 neg1 = make_float2(-1.f, -1.f);
 #pragma unroll
-  for (int i = 0; i < N; ++i) {
-    const float e = fast_exp2(fmaf(m[i], kLog2e, -md2));
-    p.s1d += e;
-    p.skd = fmaf(e, m[i] - l[i], p.skd);
-  }
-  // --- coupled Gumbel-max samples (same noise g for both)
+  for (int k = 0; k < NV; ++k)
+#pragma unroll
+    for (int e = 0; e < NP; ++e) {
+      const float2 y = __ffma2_rn(L[k][e], l2e, nmt);
+      const float2 et = ex2x2(y);
+      a.s1t = __fadd2_rn(a.s1t, et);
+      a.s2t = __ffma2_rn(et, y, a.s2t);
+      const float2 z = __ffma2_rn(M[k][e], l2e, nmd);
+      const float2 ed = ex2x2(z);
+      a.s1d = __fadd2_rn(a.s1d, ed);
+      a.skd = __ffma2_rn(ed, __ffma2_rn(L[k][e], neg1, M[k][e]), a.skd);
+    }
+  // --- coupled Gumbel-max samples (same noise for both)
   if constexpr (SAMPLE) {
-    float st[N], sd[N];
+    const float2 it2 = make_float2(invT, invT);
+    float2 ST[NV][NP], SD[NV][NP];
     float bt = -INFINITY, bd = -INFINITY;
 #pragma unroll
-    for (int i = 0; i < N; ++i) {
-      st[i] = fmaf(l[i], invT, g[i]);
-      sd[i] = fmaf(m[i], invT, g[i]);
-      bt = fmaxf(bt, st[i]);
-      bd = fmaxf(bd, sd[i]);
-    }
-    if (bt > p.bt) {
-      int a = 0;
-      float la = l[0];
+    for (int k = 0; k < NV; ++k) {
 #pragma unroll
-      for (int i = N - 1; i >= 0; --i)
-        if (st[i] == bt) { a = i; la = l[i]; }
-      p.bt = bt;
-      p.it = v0 + a;
-      p.lt_at = la;
-    }
-    if (bd > p.bd) {
-      int a = 0;
+      for (int q = 0; q < VEC / 4; ++q) {
+        const PhiloxOut o = philox4x32_10((uint32_t)(v0[k] >> 2) + q, (uint32_t)pos,
+                                          (uint32_t)b, key.step, key.k0, key.k1);
+        const float2 g01 = make_float2(gumbel_from_word(o.w[0]), gumbel_from_word(o.w[1]));
+        const float2 g23 = make_float2(gumbel_from_word(o.w[2]), gumbel_from_word(o.w[3]));
+        ST[k][2 * q] = __ffma2_rn(L[k][2 * q], it2, g01);
+        ST[k][2 * q + 1] = __ffma2_rn(L[k][2 * q + 1], it2, g23);
+        SD[k][2 * q] = __ffma2_rn(M[k][2 * q], it2, g01);
+        SD[k][2 * q + 1] = __ffma2_rn(M[k][2 * q + 1], it2, g23);
+      }
 #pragma unroll
-      for (int i = N - 1; i >= 0; --i)
-        if (sd[i] == bd) a = i;
-      p.bd = bd;
-      p.id = v0 + a;
+      for (int e = 0; e < NP; ++e) {
+        bt = fmaxf(bt, fmaxf(ST[k][e].x, ST[k][e].y));
+        bd = fmaxf(bd, fmaxf(SD[k][e].x, SD[k][e].y));
+      }
+    }
+    if (__any_sync(__activemask(), bt > a.bt) && bt > a.bt) {
+      int idx = 0x7fffffff;
+      float la = 0.f;
+#pragma unroll
+      for (int k = NV - 1; k >= 0; --k)
+#pragma unroll
+        for (int e = NP - 1; e >= 0; --e) {
+          if (ST[k][e].y == bt) { idx = v0[k] + 2 * e + 1; la = L[k][e].y; }
+          if (ST[k][e].x == bt) { idx = v0[k] + 2 * e; la = L[k][e].x; }
+        }
+      a.bt = bt;
+      a.it = idx;
+      a.lt_at = la;
+    }
+    if (__any_sync(__activemask(), bd > a.bd) && bd > a.bd) {
+      int idx = 0x7fffffff;
+#pragma unroll
+      for (int k = NV - 1; k >= 0; --k)
+#pragma unroll
+        for (int e = NP - 1; e >= 0; --e) {
+          if (SD[k][e].y == bd) idx = v0[k] + 2 * e + 1;
+          if (SD[k][e].x == bd) idx = v0[k] + 2 * e;
+        }
+      a.bd = bd;
+      a.id = idx;
     }
   }
 }
 
-// Merge partial b into a (both cover disjoint vocabulary ranges).
+// One vocabulary entry (the ragged end of a row).
+template <bool SAMPLE>
+__device__ __forceinline__ void fold_one(Acc& a, float l, float m, float g, int v, float invT) {
+  if (l > a.mt) {
+    if (a.mt != -INFINITY) {
+      const float dl = (a.mt - l) * kLog2e;
+      const float f = exp2f(dl);
+      a.s2t = make_float2(f * (a.s2t.x + dl * a.s1t.x), f * (a.s2t.y + dl * a.s1t.y));
+      a.s1t = make_float2(f * a.s1t.x, f * a.s1t.y);
+    }
+    a.mt = l;
+    a.at = v;
+  }
+  if (m > a.md) {
+    if (a.md != -INFINITY) {
+      const float f = exp2f((a.md - m) * kLog2e);
+      a.s1d = make_float2(f * a.s1d.x, f * a.s1d.y);
+      a.skd = make_float2(f * a.skd.x, f * a.skd.y);
+    }
+    a.md = m;
+    a.ad = v;
+  }
+  const float y = fmaf(l, kLog2e, -a.mt * kLog2e);
+  const float et = fast_exp2(y);
+  a.s1t.x += et;
+  a.s2t.x = fmaf(et, y, a.s2t.x);
+  const float ed = fast_exp2(fmaf(m, kLog2e, -a.md * kLog2e));
+  a.s1d.x += ed;
+  a.skd.x = fmaf(ed, m - l, a.skd.x);
+  if constexpr (SAMPLE) {
+    const float st = fmaf(l, invT, g), sd = fmaf(m, invT, g);
+    if (st > a.bt) { a.bt = st; a.it = v; a.lt_at = l; }
+    if (sd > a.bd) { a.bd = sd; a.id = v; }
+  }
+}
+
+// Merge partial b into a (both cover disjoint vocabulary ranges of one row).
 template <bool SAMPLE>
 __device__ __forceinline__ void merge(Partial& a, const Partial& b) {
-  // verifier
   if (b.mt != -INFINITY) {
     if (a.mt == -INFINITY) {
       a.mt = b.mt; a.s1t = b.s1t; a.s2t = b.s2t; a.at = b.at;
@@ -150,7 +322,6 @@ __device__ __forceinline__ void merge(Partial& a, const Partial& b) {
       a.mt = M;
     }
   }
-  // drafter
   if (b.md != -INFINITY) {
     if (a.md == -INFINITY) {
       a.md = b.md; a.s1d = b.s1d; a.skd = b.skd; a.ad = b.ad;
@@ -169,30 +340,22 @@ __device__ __forceinline__ void merge(Partial& a, const Partial& b) {
   }
 }
 
-__device__ __forceinline__ Partial shfl_down(const Partial& p, int delta) {
+__device__ __forceinline__ Partial shfl_xor(const Partial& p, int mask) {
   Partial q;
-  q.mt = __shfl_down_sync(0xffffffffu, p.mt, delta);
-  q.s1t = __shfl_down_sync(0xffffffffu, p.s1t, delta);
-  q.s2t = __shfl_down_sync(0xffffffffu, p.s2t, delta);
-  q.md = __shfl_down_sync(0xffffffffu, p.md, delta);
-  q.s1d = __shfl_down_sync(0xffffffffu, p.s1d, delta);
-  q.skd = __shfl_down_sync(0xffffffffu, p.skd, delta);
-  q.at = __shfl_down_sync(0xffffffffu, p.at, delta);
-  q.ad = __shfl_down_sync(0xffffffffu, p.ad, delta);
-  q.bt = __shfl_down_sync(0xffffffffu, p.bt, delta);
-  q.lt_at = __shfl_down_sync(0xffffffffu, p.lt_at, delta);
-  q.bd = __shfl_down_sync(0xffffffffu, p.bd, delta);
-  q.it = __shfl_down_sync(0xffffffffu, p.it, delta);
-  q.id = __shfl_down_sync(0xffffffffu, p.id, delta);
+  q.mt = __shfl_xor_sync(0xffffffffu, p.mt, mask);
+  q.s1t = __shfl_xor_sync(0xffffffffu, p.s1t, mask);
+  q.s2t = __shfl_xor_sync(0xffffffffu, p.s2t, mask);
+  q.md = __shfl_xor_sync(0xffffffffu, p.md, mask);
+  q.s1d = __shfl_xor_sync(0xffffffffu, p.s1d, mask);
+  q.skd = __shfl_xor_sync(0xffffffffu, p.skd, mask);
+  q.at = __shfl_xor_sync(0xffffffffu, p.at, mask);
+  q.ad = __shfl_xor_sync(0xffffffffu, p.ad, mask);
+  q.bt = __shfl_xor_sync(0xffffffffu, p.bt, mask);
+  q.lt_at = __shfl_xor_sync(0xffffffffu, p.lt_at, mask);
+  q.bd = __shfl_xor_sync(0xffffffffu, p.bd, mask);
+  q.it = __shfl_xor_sync(0xffffffffu, p.it, mask);
+  q.id = __shfl_xor_sync(0xffffffffu, p.id, mask);
   return q;
-}
-
-__device__ __forceinline__ uint4 ld_stream(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
 }
 
 template <typename T>
@@ -216,10 +379,6 @@ struct Vec<float> {
   __device__ static float scalar(const float* p) { return *p; }
 };
 
-struct NoiseKey {
-  uint32_t k0, k1, step;
-};
-
 // Gumbel noise of N consecutive entries starting at v0 (v0 % 4 == 0 when N >= 4).
 template <int N>
 __device__ __forceinline__ void noise(float (&g)[N], int v0, int pos, int b, const NoiseKey& key) {
@@ -237,124 +396,198 @@ __device__ __forceinline__ void noise(float (&g)[N], int v0, int pos, int b, con
       const int v = v0 + i;
       const PhiloxOut o = philox4x32_10((uint32_t)(v >> 2), (uint32_t)pos, (uint32_t)b, key.step,
                                         key.k0, key.k1);
-      g[i] = gumbel_from_word(o.w[v & 3]);
+      const uint32_t w = (v & 3) == 0 ? o.w[0] : (v & 3) == 1 ? o.w[1] : (v & 3) == 2 ? o.w[2]
+                                                                                        : o.w[3];
+      g[i] = gumbel_from_word(w);
     }
   }
 }
 
+// Work partition: U units split into G ranges, the first `rem` of size q + 1.
+struct Split {
+  int64_t q, rem;
+  __host__ __device__ int64_t begin(int64_t c) const {
+    return c < rem ? c * (q + 1) : rem * (q + 1) + (c - rem) * q;
+  }
+  __host__ __device__ int64_t size(int64_t c) const { return c < rem ? q + 1 : q; }
+  __host__ __device__ int64_t cta_of(int64_t u) const {
+    return u < rem * (q + 1) ? u / (q + 1) : rem + (u - rem * (q + 1)) / (q > 0 ? q : 1);
+  }
+};
+
+struct VerifyArgs {
+  const void *lt, *lm;
+  int R, V;
+  int64_t ld;
+  int pos_offset;
+  float invT;
+  NoiseKey key;
+  int nchunk;  // chunks per row
+  Split split;
+  Partial* parts;  // [rows, maxparts]
+  int maxparts;
+  uint32_t spin;
+};
+
+__device__ __forceinline__ uint4 ld_stream(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
 template <typename T, bool SAMPLE>
-__global__ void __launch_bounds__(kThreads)
-verify_logits_kernel(const T* __restrict__ lt, const T* __restrict__ lm, int R, int V,
-                     int64_t ld, int pos_offset, float invT, NoiseKey key, int seg_len,
-                     dd_row_stats out) {
+__global__ void __launch_bounds__(kVThreads, VCfg<SAMPLE>::kMinBlocks)
+verify_stream_kernel(const VerifyArgs a) {
   constexpr int VEC = Vec<T>::N;
-  cg::cluster_group cluster = cg::this_cluster();
-  const int C = (int)cluster.num_blocks();
-  const int rank = (int)cluster.block_rank();
-  const int row = blockIdx.x / C;
-  const int b = row / R;
-  const int pos = pos_offset + row % R;
-  const int seg0 = rank * seg_len;
-  const int seg1 = min(V, seg0 + seg_len);
-  const T* lrow = lt + (int64_t)row * ld;
-  const T* mrow = lm + (int64_t)row * ld;
+  __shared__ Partial red[kVThreads / 32];
 
-  Partial p;
-  init(p);
-  float gz[VEC];
-#pragma unroll
-  for (int i = 0; i < VEC; ++i) gz[i] = 0.f;
+  const int c = blockIdx.x;
+  const int ct = threadIdx.x, lane = ct & 31, cw = ct >> 5;
+  const T* LT = static_cast<const T*>(a.lt);
+  const T* LM = static_cast<const T*>(a.lm);
+  const int spr = a.nchunk;                       // vector slots per row
+  const int nvr = (int)(((int64_t)a.V * (int)sizeof(T)) >> 4);  // full vectors per row
+  const int64_t s0 = a.split.begin(c), s1 = s0 + a.split.size(c);
 
-  if (seg0 < seg1) {
-    const int nvec = (seg1 - seg0) / VEC;  // full vectors (seg0 is a multiple of 64)
-    const uint4* lv = reinterpret_cast<const uint4*>(lrow + seg0);
-    const uint4* mv = reinterpret_cast<const uint4*>(mrow + seg0);
-    for (int base = threadIdx.x; base < nvec; base += kUnroll * kThreads) {
-      uint4 a[kUnroll], c[kUnroll];
+  Acc acc;
+  init(acc);
+  auto flush = [&](int64_t row) {
+    Partial p = to_partial(acc);
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int idx = base + u * kThreads;
-        if (idx < nvec) { a[u] = ld_stream(lv + idx); c[u] = ld_stream(mv + idx); }
+    for (int mask = 16; mask > 0; mask >>= 1) {
+      const Partial q = shfl_xor(p, mask);
+      merge<SAMPLE>(p, q);
+    }
+    if (lane == 0) red[cw] = p;
+    __syncthreads();
+    if (cw == 0) {
+      Partial r;
+      if (lane < kVThreads / 32) {
+        r = red[lane];
+      } else {
+        Acc e;
+        init(e);
+        r = to_partial(e);
       }
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int idx = base + u * kThreads;
-        if (idx < nvec) {
-          float x[VEC], y[VEC];
-          Vec<T>::unpack(a[u], x);
-          Vec<T>::unpack(c[u], y);
-          const int v0 = seg0 + idx * VEC;
-          if constexpr (SAMPLE) {
-            float g[VEC];
-            noise<VEC>(g, v0, pos, b, key);
-            accumulate<VEC, SAMPLE>(p, x, y, g, v0, invT);
-          } else {
-            accumulate<VEC, SAMPLE>(p, x, y, gz, v0, invT);
-          }
+      for (int mask = 16; mask > 0; mask >>= 1) {
+        const Partial q = shfl_xor(r, mask);
+        merge<SAMPLE>(r, q);
+      }
+      if (lane == 0) {
+        const int64_t slot = c - a.split.cta_of(row * spr);
+        a.parts[row * a.maxparts + slot] = r;
+      }
+    }
+    __syncthreads();
+    init(acc);
+  };
+
+  for (int64_t sidx = s0; sidx < s1;) {
+    const int64_t row = sidx / spr;
+    const int vbeg = (int)(sidx - row * spr);
+    const int64_t rest = s1 - sidx;
+    const int vend = rest < (int64_t)(spr - vbeg) ? vbeg + (int)rest : spr;
+    const int b = (int)(row / a.R);
+    const int pos = a.pos_offset + (int)(row - (int64_t)b * a.R);
+    const uint4* lv = reinterpret_cast<const uint4*>(LT + row * a.ld);
+    const uint4* mv = reinterpret_cast<const uint4*>(LM + row * a.ld);
+    const int vlim = min(vend, nvr);  // slots past nvr carry no full vector
+    // Two vectors per matrix per half-step; while one pair is folded the next
+    // pair's loads are in flight (ping-pong, no register moves).
+    auto ld2 = [&](int bs, uint4 (&l)[2], uint4 (&m)[2]) {
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int idx = bs + k * kVThreads;
+        if (idx < vlim) {
+          l[k] = ld_stream(lv + idx);
+          m[k] = ld_stream(mv + idx);
         }
       }
-    }
-    // ragged tail of the row (fewer than VEC entries), one entry per thread
-    const int tail0 = seg0 + nvec * VEC;
-    const int v = tail0 + threadIdx.x;
-    if (v < seg1) {
-      float x[1] = {Vec<T>::scalar(lrow + v)};
-      float y[1] = {Vec<T>::scalar(mrow + v)};
-      float g[1] = {0.f};
-      if constexpr (SAMPLE) noise<1>(g, v, pos, b, key);
-      accumulate<1, SAMPLE>(p, x, y, g, v, invT);
-    }
-  }
-
-  // --- CTA reduction: warp shuffles, then across warps through shared memory
+    };
+    auto fold2 = [&](int bs, const uint4 (&l)[2], const uint4 (&m)[2]) {
 #pragma unroll
-  for (int delta = 16; delta > 0; delta >>= 1) {
-    const Partial q = shfl_down(p, delta);
-    merge<SAMPLE>(p, q);
-  }
-  __shared__ Partial warp_part[kThreads / 32];
-  __shared__ Partial cta_part;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (lane == 0) warp_part[warp] = p;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    Partial acc = warp_part[0];
-    for (int w = 1; w < kThreads / 32; ++w) merge<SAMPLE>(acc, warp_part[w]);
-    cta_part = acc;
-  }
-  // --- cluster reduction through distributed shared memory
-  cluster.sync();
-  if (rank == 0 && threadIdx.x == 0) {
-    Partial acc = cta_part;
-    for (int r = 1; r < C; ++r) {
-      const Partial* remote = cluster.map_shared_rank(&cta_part, r);
-      merge<SAMPLE>(acc, *remote);
+      for (int k = 0; k < 2; ++k) {
+        const int idx = bs + k * kVThreads;
+        if (idx < vlim) {
+          uint4 l1[1] = {l[k]}, m1[1] = {m[k]};
+          int vv[1] = {idx * VEC};
+          fold<T, SAMPLE, 1>(acc, l1, m1, vv, pos, b, a.key, a.invT);
+        }
+      }
+    };
+    constexpr int kStep = 2 * kVThreads;
+    uint4 la[2], ma[2], lb[2], mb[2];
+    int base = vbeg + ct;
+    ld2(base, la, ma);
+    for (; base < vlim; base += 2 * kStep) {
+      ld2(base + kStep, lb, mb);
+      fold2(base, la, ma);
+      ld2(base + 2 * kStep, la, ma);
+      fold2(base + kStep, lb, mb);
     }
-    const float ln_s1t = logf(acc.s1t);
-    const float lse_t = acc.mt + ln_s1t;
-    const float lse_d = acc.md + logf(acc.s1d);
-    const float conf = 1.f / acc.s1t;
-    const float ent = ln_s1t - acc.s2t * kLn2 / acc.s1t;
-    const float kl = acc.skd / acc.s1d + (acc.mt - acc.md) + logf(acc.s1t / acc.s1d);
-    int st = acc.at, sd = acc.ad;
-    float psamp = conf;
-    if constexpr (SAMPLE) {
-      st = acc.it;
-      sd = acc.id;
-      psamp = expf(acc.lt_at - lse_t);
+    if (vend == spr) {
+      // ragged end of the row (fewer than 16 bytes): one entry per thread
+      const int e = nvr * VEC + ct;
+      if (e < a.V) {
+        float g = 0.f;
+        if constexpr (SAMPLE) {
+          float gg[1];
+          noise<1>(gg, e, pos, b, a.key);
+          g = gg[0];
+        }
+        fold_one<SAMPLE>(acc, Vec<T>::scalar(LT + row * a.ld + e),
+                         Vec<T>::scalar(LM + row * a.ld + e), g, e, a.invT);
+      }
     }
-    if (out.lse_t) out.lse_t[row] = lse_t;
-    if (out.lse_d) out.lse_d[row] = lse_d;
-    if (out.conf_t) out.conf_t[row] = conf;
-    if (out.p_sample_t) out.p_sample_t[row] = psamp;
-    if (out.entropy_t) out.entropy_t[row] = ent;
-    if (out.kl_dt) out.kl_dt[row] = kl;
-    if (out.argmax_t) out.argmax_t[row] = acc.at;
-    if (out.argmax_d) out.argmax_d[row] = acc.ad;
-    if (out.sample_t) out.sample_t[row] = st;
-    if (out.sample_d) out.sample_d[row] = sd;
+    flush(row);
+    sidx += vend - vbeg;
   }
-  cluster.sync();  // keep every CTA's shared memory alive until rank 0 has read it
+}
+
+// One warp per row: merge the row's partials and write the statistics.
+template <bool SAMPLE>
+__global__ void __launch_bounds__(256) verify_merge_kernel(const VerifyArgs a, int rows,
+                                                           dd_row_stats out) {
+  const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const int64_t c0 = a.split.cta_of(row * a.nchunk);
+  const int nparts = (int)(a.split.cta_of(row * a.nchunk + a.nchunk - 1) - c0 + 1);
+  Partial acc;
+  init(acc);
+  for (int k = lane; k < nparts; k += 32) merge<SAMPLE>(acc, a.parts[row * a.maxparts + k]);
+#pragma unroll
+  for (int mask = 16; mask > 0; mask >>= 1) {
+    const Partial q = shfl_xor(acc, mask);
+    merge<SAMPLE>(acc, q);
+  }
+  if (lane != 0) return;
+  const float ln_s1t = logf(acc.s1t);
+  const float lse_t = acc.mt + ln_s1t;
+  const float lse_d = acc.md + logf(acc.s1d);
+  const float conf = 1.f / acc.s1t;
+  const float ent = ln_s1t - acc.s2t * kLn2 / acc.s1t;
+  const float kl = acc.skd / acc.s1d + (acc.mt - acc.md) + logf(acc.s1t / acc.s1d);
+  int st = acc.at, sd = acc.ad;
+  float psamp = conf;
+  if constexpr (SAMPLE) {
+    st = acc.it;
+    sd = acc.id;
+    psamp = expf(acc.lt_at - lse_t);
+  }
+  if (out.lse_t) out.lse_t[row] = lse_t;
+  if (out.lse_d) out.lse_d[row] = lse_d;
+  if (out.conf_t) out.conf_t[row] = conf;
+  if (out.p_sample_t) out.p_sample_t[row] = psamp;
+  if (out.entropy_t) out.entropy_t[row] = ent;
+  if (out.kl_dt) out.kl_dt[row] = kl;
+  if (out.argmax_t) out.argmax_t[row] = acc.at;
+  if (out.argmax_d) out.argmax_d[row] = acc.ad;
+  if (out.sample_t) out.sample_t[row] = st;
+  if (out.sample_d) out.sample_d[row] = sd;
 }
 
 __global__ void coupled_gumbel_kernel(NoiseKey key, int R, int V, int64_t ld, int pos_offset,
@@ -374,62 +607,88 @@ __global__ void coupled_gumbel_kernel(NoiseKey key, int R, int V, int64_t ld, in
   }
 }
 
+// Grid and partition for a call (also sizes the workspace).
+struct VerifyPlan {
+  int grid, nchunk, maxparts;
+  Split split;
+};
+
+VerifyPlan plan_verify(int rows, int V, int esize, int sm_count, int per_sm) {
+  VerifyPlan pl;
+  const int64_t nvr = ((int64_t)V * esize) >> 4;
+  pl.nchunk = (int)(nvr > 0 ? nvr : 1);  // vector slots per row
+  const int64_t units = (int64_t)rows * pl.nchunk;
+  // at least 2048 vectors per CTA, so a piece is long enough to stream
+  int64_t g = (int64_t)sm_count * per_sm;
+  const int64_t gmin = (units + 2047) / 2048;
+  if (g > gmin) g = gmin > 0 ? gmin : 1;
+  pl.grid = (int)g;
+  pl.split.q = units / pl.grid;
+  pl.split.rem = units % pl.grid;
+  // a row's slots overlap at most ceil(nchunk / q) + 1 ranges
+  const int64_t q = pl.split.q > 0 ? pl.split.q : 1;
+  pl.maxparts = (int)((pl.nchunk + q - 1) / q + 1);
+  return pl;
+}
+
+// The workspace bound must hold on any device: plan for up to 512 SMs.
+constexpr int kPlanSmBound = 512;
+
 template <typename T, bool SAMPLE>
 cudaError_t launch_verify(const void* lt, const void* lm, int B, int R, int V, int64_t ld,
                           int pos_offset, float temperature, NoiseKey key,
-                          const dd_row_stats& out, cudaStream_t stream) {
-  auto kern = verify_logits_kernel<T, SAMPLE>;
+                          const dd_row_stats& out, void* workspace, cudaStream_t stream) {
   const int rows = B * R;
   const DeviceInfo& dev = device_info();
-  int per_sm = 0;
-  cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, 0);
+  VerifyPlan pl = plan_verify(rows, V, (int)sizeof(T), dev.sm_count, VCfg<SAMPLE>::kMinBlocks);
+  const VerifyPlan bound = plan_verify(rows, V, (int)sizeof(T), kPlanSmBound, kMaxGridPerSm);
+  VerifyArgs a;
+  a.lt = lt;
+  a.lm = lm;
+  a.R = R;
+  a.V = V;
+  a.ld = ld;
+  a.pos_offset = pos_offset;
+  a.invT = temperature > 0.f ? 1.f / temperature : 0.f;
+  a.key = key;
+  a.nchunk = pl.nchunk;
+  a.split = pl.split;
+  a.parts = static_cast<Partial*>(workspace);
+  a.maxparts = bound.maxparts > pl.maxparts ? bound.maxparts : pl.maxparts;
+  a.spin = spin_limit();
+  verify_stream_kernel<T, SAMPLE><<<pl.grid, kVThreads, 0, stream>>>(a);
+  cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  const int64_t slots = (int64_t)dev.sm_count * (per_sm > 0 ? per_sm : 1);
-  // Split rows into C segments (a power of two <= 8) while the whole grid
-  // still fits in one wave and every thread keeps at least 2 vectors per matrix.
-  constexpr int VEC = Vec<T>::N;
-  int C = 1;
-  while (C < 8 && (int64_t)rows * (2 * C) <= slots &&
-         (int64_t)V >= (int64_t)(2 * C) * kThreads * VEC * 2)
-    C *= 2;
-  int seg_len = (V + C - 1) / C;
-  seg_len = (seg_len + 63) / 64 * 64;
-
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(rows * C), 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = C;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  const float invT = temperature > 0.f ? 1.f / temperature : 0.f;
-  return cudaLaunchKernelEx(&cfg, kern, static_cast<const T*>(lt), static_cast<const T*>(lm), R,
-                            V, ld, pos_offset, invT, key, seg_len, out);
+  verify_merge_kernel<SAMPLE><<<(rows + 7) / 8, 256, 0, stream>>>(a, rows, out);
+  return cudaGetLastError();
 }
 
 }  // namespace
 
+size_t verify_workspace_bytes(int B, int R, int V, dd_dtype dtype) {
+  const int esize = dtype == DD_BF16 ? 2 : 4;
+  const int rows = B * R;
+  const VerifyPlan bound = plan_verify(rows, V, esize, kPlanSmBound, kMaxGridPerSm);
+  // any real device has at most kPlanSmBound SMs, so its maxparts is no larger
+  return (size_t)rows * bound.maxparts * sizeof(Partial);
+}
+
 cudaError_t launch_verify_logits(const void* lt, const void* lm, dd_dtype dtype, int B, int R,
                                  int V, int64_t ld, int pos_offset, float temperature,
                                  uint64_t seed, uint64_t step, const dd_row_stats& out,
-                                 cudaStream_t stream) {
+                                 void* workspace, cudaStream_t stream) {
   NoiseKey key{(uint32_t)(seed & 0xffffffffu), (uint32_t)(seed >> 32),
                (uint32_t)(step & 0xffffffffu)};
   const bool sample = temperature > 0.f;
   if (dtype == DD_BF16)
     return sample ? launch_verify<__nv_bfloat16, true>(lt, lm, B, R, V, ld, pos_offset,
-                                                       temperature, key, out, stream)
+                                                       temperature, key, out, workspace, stream)
                   : launch_verify<__nv_bfloat16, false>(lt, lm, B, R, V, ld, pos_offset,
-                                                        temperature, key, out, stream);
+                                                        temperature, key, out, workspace, stream);
   return sample ? launch_verify<float, true>(lt, lm, B, R, V, ld, pos_offset, temperature, key,
-                                             out, stream)
+                                             out, workspace, stream)
                 : launch_verify<float, false>(lt, lm, B, R, V, ld, pos_offset, temperature, key,
-                                              out, stream);
+                                              out, workspace, stream);
 }
 
 cudaError_t launch_coupled_gumbel(uint64_t seed, uint64_t step, int B, int R, int V, int64_t ld,

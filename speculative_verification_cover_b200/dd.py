@@ -25,6 +25,7 @@ DD_MASK_TOKEN = -1
 # Every symbol include/dd.h declares.
 EXPORTED = (
     "dd_dualview_attention", "dd_dualview_attention_workspace_size", "dd_verify_logits",
+    "dd_verify_logits_workspace_size",
     "dd_coupled_gumbel", "dd_select_seeds", "dd_decide", "dd_status_string",
     "dd_get_device_error", "dd_set_spin_limit", "dd_selftest_bounded_wait",
 )
@@ -66,8 +67,10 @@ def lib():
     L.dd_dualview_attention_workspace_size.argtypes = [I] * 5
     L.dd_dualview_attention_workspace_size.restype = SZ
     L.dd_verify_logits.argtypes = [P, P, I, I, I, I, I64, I, F, U64, U64,
-                                   ctypes.POINTER(_RowStats), P]
+                                   ctypes.POINTER(_RowStats), P, SZ, P]
     L.dd_verify_logits.restype = I
+    L.dd_verify_logits_workspace_size.argtypes = [I, I, I, I]
+    L.dd_verify_logits_workspace_size.restype = SZ
     L.dd_coupled_gumbel.argtypes = [U64, U64, I, I, I, I64, I, P, P]
     L.dd_coupled_gumbel.restype = I
     L.dd_select_seeds.argtypes = [P, I, I, P, P, P, I, I, I, P, P, P, P]
@@ -170,11 +173,21 @@ def dd_dualview_attention(q, k_cur, v_cur, k_prev, v_prev, is_seed, is_masked, i
     _check("dd_dualview_attention", st)
 
 
+def dd_verify_logits_workspace_size(B, R, V, dtype) -> int:
+    code = dtype if isinstance(dtype, int) else _dtype_code(torch.empty(0, dtype=dtype))
+    return int(lib().dd_verify_logits_workspace_size(B, R, V, code))
+
+
 def dd_verify_logits(logits_t, logits_d, out: RowStats, pos_offset=0, temperature=0.0, seed=0,
-                     step=0, stream=None):
+                     step=0, workspace=None, stream=None):
     """logits [B,R,V]; a view narrowed from a wider [B,R,ld] buffer is accepted
-    (the row stride ld is read from the tensor). out: RowStats of [B,R] tensors."""
+    (the row stride ld is read from the tensor). out: RowStats of [B,R] tensors.
+    workspace: uint8 device tensor of dd_verify_logits_workspace_size(...) bytes
+    (allocated here with torch when not given)."""
     B, R, V = logits_t.shape
+    if workspace is None:
+        workspace = torch.empty(dd_verify_logits_workspace_size(B, R, V, logits_t.dtype),
+                                dtype=torch.uint8, device=logits_t.device)
     if logits_t.stride(2) != 1 or logits_t.stride(0) != R * logits_t.stride(1):
         raise ValueError("logits must be [B,R,V] with unit vocabulary stride and packed rows")
     if logits_d.shape != logits_t.shape or logits_d.stride() != logits_t.stride():
@@ -186,7 +199,7 @@ def dd_verify_logits(logits_t, logits_d, out: RowStats, pos_offset=0, temperatur
         ctypes.c_void_p(logits_t.data_ptr()), ctypes.c_void_p(logits_d.data_ptr()),
         _dtype_code(logits_t), B, R, V, ld, int(pos_offset), float(temperature),
         int(seed) & (2**64 - 1), int(step) & (2**64 - 1), ctypes.byref(out._c()),
-        _stream(stream))
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
     _check("dd_verify_logits", st)
 
 

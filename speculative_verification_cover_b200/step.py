@@ -17,8 +17,8 @@ from .workloads import WorkloadSpec
 
 INPUT_KEYS = ("q", "k_cur", "v_cur", "k_prev", "v_prev", "is_seed", "is_masked", "is_new",
               "eligible", "tokens", "logits_t", "logits_d")
-# Our kernels per step: masked-row compaction, attention pass 1, pass 2, two
-# head reductions, verify, select, decide.
+# Our kernels per step: mask preparation, attention pass 1, pass 2, head
+# reduction, vocabulary stream + merge, seed selection, decisions.
 KERNELS_PER_STEP = 8
 
 
@@ -38,6 +38,9 @@ class VerifyStep:
         self.ws = torch.empty(dd.dd_dualview_attention_workspace_size(B, L, Hq, Hkv, d),
                               dtype=torch.uint8, device=dev)
         self.stats = dd.RowStats.empty(B, R, dev)
+        self.vws = torch.empty(dd.dd_verify_logits_workspace_size(B, R, spec.V,
+                                                                  self.x["logits_t"].dtype),
+                               dtype=torch.uint8, device=dev)
         self.k = max(spec.k, 1)
         self.next_seeds = torch.empty(B, self.k, dtype=torch.int32, device=dev)
         self.next_is_seed = torch.empty(B, L, dtype=torch.uint8, device=dev)
@@ -59,7 +62,7 @@ class VerifyStep:
         s = self.spec
         dd.dd_verify_logits(self.x["logits_t"], self.x["logits_d"], self.stats,
                             pos_offset=s.pos_offset, temperature=s.temperature, seed=self.seed,
-                            step=self.step_index)
+                            step=self.step_index, workspace=self.vws)
 
     def select_and_decide(self):
         s, x = self.spec, self.x

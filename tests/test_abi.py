@@ -88,8 +88,10 @@ def _verify(lib, **over):
     a = dict(lt=FAKE, lm=FAKE, dtype=1, B=1, R=4, V=100, ld=104, off=0, T=0.0)
     a.update(over)
     stats = dd._RowStats()
+    ws = a.get("ws", P(0x100000))
+    wsb = a.get("wsb", 1 << 20)
     return lib.dd_verify_logits(a["lt"], a["lm"], a["dtype"], a["B"], a["R"], a["V"], a["ld"],
-                                a["off"], a["T"], 0, 0, ctypes.byref(stats), None)
+                                a["off"], a["T"], 0, 0, ctypes.byref(stats), ws, wsb, None)
 
 
 def test_verify_validation(lib):
@@ -101,8 +103,14 @@ def test_verify_validation(lib):
     assert _verify(lib, T=float("inf")) == dd.DD_ERR_INVALID_ARG
     assert _verify(lib, lm=MISALIGNED) == dd.DD_ERR_INVALID_ARG
     assert _verify(lib, dtype=0, ld=102) == dd.DD_ERR_INVALID_ARG   # fp32: 408 bytes
-    assert lib.dd_verify_logits(FAKE, FAKE, 1, 1, 4, 100, 104, 0, 0.0, 0, 0, None, None) \
-        == dd.DD_ERR_INVALID_ARG
+    assert lib.dd_verify_logits(FAKE, FAKE, 1, 1, 4, 100, 104, 0, 0.0, 0, 0, None, P(0x100000),
+                                1 << 20, None) == dd.DD_ERR_INVALID_ARG
+    assert _verify(lib, ws=None) == dd.DD_ERR_INVALID_ARG
+    assert _verify(lib, wsb=16) == dd.DD_ERR_INVALID_ARG
+    assert _verify(lib, ws=P(0x100010)) == dd.DD_ERR_INVALID_ARG    # not 256-aligned
+    n = dd.dd_verify_logits_workspace_size(16, 768, 126464, 1)
+    assert n > 0 and n % 64 == 0
+    assert dd.dd_verify_logits_workspace_size(0, 768, 126464, 1) == 0
 
 
 def test_select_and_decide_validation(lib):
