@@ -58,42 +58,51 @@ __device__ __forceinline__ void init(Partial& p) {
   p.it = p.id = 0x7fffffff;
 }
 
+template <typename T>
+struct Vec;
+template <>
+struct Vec<__nv_bfloat16> {
+  static constexpr int N = 8;
+  __device__ static void unpack(const uint4& u, float (&x)[8]) {
+    x[0] = bf16lo(u.x); x[1] = bf16hi(u.x); x[2] = bf16lo(u.y); x[3] = bf16hi(u.y);
+    x[4] = bf16lo(u.z); x[5] = bf16hi(u.z); x[6] = bf16lo(u.w); x[7] = bf16hi(u.w);
+  }
+  __device__ static float scalar(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+};
+template <>
+struct Vec<float> {
+  static constexpr int N = 4;
+  __device__ static void unpack(const uint4& u, float (&x)[4]) {
+    x[0] = __uint_as_float(u.x); x[1] = __uint_as_float(u.y);
+    x[2] = __uint_as_float(u.z); x[3] = __uint_as_float(u.w);
+  }
+  __device__ static float scalar(const float* p) { return *p; }
+};
+
 // Per-thread accumulator: the sums are float2 so that pairs of vocabulary
 // entries go through the packed fp32 pipe (FFMA2 / FADD2) and each sum has two
-// independent dependency chains.
+// independent dependency chains. The exponentials are taken against a
+// reference (ref_t / ref_d) that is moved only when the running maximum grows
+// by more than kRefMargin, so rescaling is rare; the exact maxima (mt / md) and
+// the 16-byte vector where each first appeared (vt / vd) are tracked with two
+// selects, and the element index inside that vector is recovered at flush time.
+// A negative vt / vd encodes an exact element index (-1 - index).
+constexpr float kRefMargin = 20.f;  // e^20 headroom: sums stay far from fp32 overflow
+
 struct Acc {
-  float mt, md;
+  float mt, md;        // exact running maxima of l and m
+  float ref_t, ref_d;  // exponent references
   float2 s1t, s2t, s1d, skd;
-  int at, ad;
-  float bt, lt_at, bd;
-  int it, id;
+  int vt, vd;          // where the maxima were first seen
+  float bt, bd;        // best coupled scores
+  int vbt, vbd;        // where they were first seen
 };
 
 __device__ __forceinline__ void init(Acc& a) {
-  a.mt = a.md = -INFINITY;
+  a.mt = a.md = a.ref_t = a.ref_d = -INFINITY;
   a.s1t = a.s2t = a.s1d = a.skd = make_float2(0.f, 0.f);
-  a.at = a.ad = 0x7fffffff;
+  a.vt = a.vd = a.vbt = a.vbd = 0x7fffffff;
   a.bt = a.bd = -INFINITY;
-  a.lt_at = 0.f;
-  a.it = a.id = 0x7fffffff;
-}
-
-__device__ __forceinline__ Partial to_partial(const Acc& a) {
-  Partial p;
-  p.mt = a.mt;
-  p.s1t = a.s1t.x + a.s1t.y;
-  p.s2t = a.s2t.x + a.s2t.y;
-  p.md = a.md;
-  p.s1d = a.s1d.x + a.s1d.y;
-  p.skd = a.skd.x + a.skd.y;
-  p.at = a.at;
-  p.ad = a.ad;
-  p.bt = a.bt;
-  p.lt_at = a.lt_at;
-  p.bd = a.bd;
-  p.it = a.it;
-  p.id = a.id;
-  return p;
 }
 
 __device__ __forceinline__ float2 ex2x2(float2 y) {
@@ -154,55 +163,43 @@ __device__ __forceinline__ void fold(Acc& a, const uint4 (&lw)[NV], const uint4 
     Unpack<T>::run(lw[k], L[k]);
     Unpack<T>::run(mw[k], M[k]);
   }
-  // --- maxima; a new maximum (rare after the first few vectors) rescales the sums
+  // --- exact maxima and the first vector holding them (selects, no branch)
   float cm = Unpack<T>::vmax(lw[0]), dm = Unpack<T>::vmax(mw[0]);
+  int cv = v0[0], dv = v0[0];
 #pragma unroll
   for (int k = 1; k < NV; ++k) {
-    cm = fmaxf(cm, Unpack<T>::vmax(lw[k]));
-    dm = fmaxf(dm, Unpack<T>::vmax(mw[k]));
+    const float x = Unpack<T>::vmax(lw[k]), y = Unpack<T>::vmax(mw[k]);
+    if (x > cm) { cm = x; cv = v0[k]; }
+    if (y > dm) { dm = y; dv = v0[k]; }
   }
-  // A new maximum is rare after the first vectors of a row: branch on a warp
-  // vote so the rescale / argmax scan is skipped, not executed predicated.
-  if (__any_sync(__activemask(), cm > a.mt) && cm > a.mt) {
-    int idx = 0x7fffffff;
-#pragma unroll
-    for (int k = NV - 1; k >= 0; --k)
-#pragma unroll
-      for (int e = NP - 1; e >= 0; --e) {
-        if (L[k][e].y == cm) idx = v0[k] + 2 * e + 1;
-        if (L[k][e].x == cm) idx = v0[k] + 2 * e;
+  if (cm > a.mt) { a.mt = cm; a.vt = cv; }
+  if (dm > a.md) { a.md = dm; a.vd = dv; }
+  // --- move an exponent reference only when its maximum outgrew it (rare)
+  const bool rt = a.mt > a.ref_t + kRefMargin, rd = a.md > a.ref_d + kRefMargin;
+  if (__any_sync(__activemask(), rt || rd)) {
+    if (rt) {
+      if (a.ref_t != -INFINITY) {
+        const float dl = (a.ref_t - a.mt) * kLog2e;
+        const float f = exp2f(dl);
+        const float2 f2 = make_float2(f, f), dl2 = make_float2(dl, dl);
+        a.s2t = __fmul2_rn(f2, __ffma2_rn(dl2, a.s1t, a.s2t));
+        a.s1t = __fmul2_rn(f2, a.s1t);
       }
-    if (a.mt != -INFINITY) {
-      const float dl = (a.mt - cm) * kLog2e;
-      const float f = exp2f(dl);
-      const float2 f2 = make_float2(f, f), dl2 = make_float2(dl, dl);
-      a.s2t = __fmul2_rn(f2, __ffma2_rn(dl2, a.s1t, a.s2t));
-      a.s1t = __fmul2_rn(f2, a.s1t);
+      a.ref_t = a.mt;
     }
-    a.mt = cm;
-    a.at = idx;
-  }
-  if (__any_sync(__activemask(), dm > a.md) && dm > a.md) {
-    int idx = 0x7fffffff;
-#pragma unroll
-    for (int k = NV - 1; k >= 0; --k)
-#pragma unroll
-      for (int e = NP - 1; e >= 0; --e) {
-        if (M[k][e].y == dm) idx = v0[k] + 2 * e + 1;
-        if (M[k][e].x == dm) idx = v0[k] + 2 * e;
+    if (rd) {
+      if (a.ref_d != -INFINITY) {
+        const float f = exp2f((a.ref_d - a.md) * kLog2e);
+        const float2 f2 = make_float2(f, f);
+        a.s1d = __fmul2_rn(f2, a.s1d);
+        a.skd = __fmul2_rn(f2, a.skd);
       }
-    if (a.md != -INFINITY) {
-      const float f = exp2f((a.md - dm) * kLog2e);
-      const float2 f2 = make_float2(f, f);
-      a.s1d = __fmul2_rn(f2, a.s1d);
-      a.skd = __fmul2_rn(f2, a.skd);
+      a.ref_d = a.md;
     }
-    a.md = dm;
-    a.ad = idx;
   }
   const float2 l2e = make_float2(kLog2e, kLog2e);
-  const float2 nmt = make_float2(-a.mt * kLog2e, -a.mt * kLog2e);
-  const float2 nmd = make_float2(-a.md * kLog2e, -a.md * kLog2e);
+  const float2 nmt = make_float2(-a.ref_t * kLog2e, -a.ref_t * kLog2e);
+  const float2 nmd = make_float2(-a.ref_d * kLog2e, -a.ref_d * kLog2e);
   const float2 neg1 = make_float2(-1.f, -1.f);
 #pragma unroll
   for (int k = 0; k < NV; ++k)
@@ -217,93 +214,136 @@ __device__ __forceinline__ void fold(Acc& a, const uint4 (&lw)[NV], const uint4 
       a.s1d = __fadd2_rn(a.s1d, ed);
       a.skd = __ffma2_rn(ed, __ffma2_rn(L[k][e], neg1, M[k][e]), a.skd);
     }
-  // --- coupled Gumbel-max samples (same noise for both)
+  // --- coupled Gumbel-max samples (same noise for both); best score + its vector
   if constexpr (SAMPLE) {
     const float2 it2 = make_float2(invT, invT);
-    float2 ST[NV][NP], SD[NV][NP];
-    float bt = -INFINITY, bd = -INFINITY;
 #pragma unroll
     for (int k = 0; k < NV; ++k) {
+      float bt = -INFINITY, bd = -INFINITY;
 #pragma unroll
       for (int q = 0; q < VEC / 4; ++q) {
         const PhiloxOut o = philox4x32_10((uint32_t)(v0[k] >> 2) + q, (uint32_t)pos,
                                           (uint32_t)b, key.step, key.k0, key.k1);
         const float2 g01 = make_float2(gumbel_from_word(o.w[0]), gumbel_from_word(o.w[1]));
         const float2 g23 = make_float2(gumbel_from_word(o.w[2]), gumbel_from_word(o.w[3]));
-        ST[k][2 * q] = __ffma2_rn(L[k][2 * q], it2, g01);
-        ST[k][2 * q + 1] = __ffma2_rn(L[k][2 * q + 1], it2, g23);
-        SD[k][2 * q] = __ffma2_rn(M[k][2 * q], it2, g01);
-        SD[k][2 * q + 1] = __ffma2_rn(M[k][2 * q + 1], it2, g23);
+        const float2 s0 = __ffma2_rn(L[k][2 * q], it2, g01);
+        const float2 s1 = __ffma2_rn(L[k][2 * q + 1], it2, g23);
+        const float2 d0 = __ffma2_rn(M[k][2 * q], it2, g01);
+        const float2 d1 = __ffma2_rn(M[k][2 * q + 1], it2, g23);
+        bt = fmaxf(bt, fmaxf(fmaxf(s0.x, s0.y), fmaxf(s1.x, s1.y)));
+        bd = fmaxf(bd, fmaxf(fmaxf(d0.x, d0.y), fmaxf(d1.x, d1.y)));
       }
-#pragma unroll
-      for (int e = 0; e < NP; ++e) {
-        bt = fmaxf(bt, fmaxf(ST[k][e].x, ST[k][e].y));
-        bd = fmaxf(bd, fmaxf(SD[k][e].x, SD[k][e].y));
-      }
-    }
-    if (__any_sync(__activemask(), bt > a.bt) && bt > a.bt) {
-      int idx = 0x7fffffff;
-      float la = 0.f;
-#pragma unroll
-      for (int k = NV - 1; k >= 0; --k)
-#pragma unroll
-        for (int e = NP - 1; e >= 0; --e) {
-          if (ST[k][e].y == bt) { idx = v0[k] + 2 * e + 1; la = L[k][e].y; }
-          if (ST[k][e].x == bt) { idx = v0[k] + 2 * e; la = L[k][e].x; }
-        }
-      a.bt = bt;
-      a.it = idx;
-      a.lt_at = la;
-    }
-    if (__any_sync(__activemask(), bd > a.bd) && bd > a.bd) {
-      int idx = 0x7fffffff;
-#pragma unroll
-      for (int k = NV - 1; k >= 0; --k)
-#pragma unroll
-        for (int e = NP - 1; e >= 0; --e) {
-          if (SD[k][e].y == bd) idx = v0[k] + 2 * e + 1;
-          if (SD[k][e].x == bd) idx = v0[k] + 2 * e;
-        }
-      a.bd = bd;
-      a.id = idx;
+      if (bt > a.bt) { a.bt = bt; a.vbt = v0[k]; }
+      if (bd > a.bd) { a.bd = bd; a.vbd = v0[k]; }
     }
   }
 }
 
-// One vocabulary entry (the ragged end of a row).
+// One vocabulary entry (the ragged end of a row); exact indices encoded -1 - v.
 template <bool SAMPLE>
 __device__ __forceinline__ void fold_one(Acc& a, float l, float m, float g, int v, float invT) {
-  if (l > a.mt) {
-    if (a.mt != -INFINITY) {
-      const float dl = (a.mt - l) * kLog2e;
+  if (l > a.mt) { a.mt = l; a.vt = -1 - v; }
+  if (m > a.md) { a.md = m; a.vd = -1 - v; }
+  if (a.mt > a.ref_t + kRefMargin) {
+    if (a.ref_t != -INFINITY) {
+      const float dl = (a.ref_t - a.mt) * kLog2e;
       const float f = exp2f(dl);
       a.s2t = make_float2(f * (a.s2t.x + dl * a.s1t.x), f * (a.s2t.y + dl * a.s1t.y));
       a.s1t = make_float2(f * a.s1t.x, f * a.s1t.y);
     }
-    a.mt = l;
-    a.at = v;
+    a.ref_t = a.mt;
   }
-  if (m > a.md) {
-    if (a.md != -INFINITY) {
-      const float f = exp2f((a.md - m) * kLog2e);
+  if (a.md > a.ref_d + kRefMargin) {
+    if (a.ref_d != -INFINITY) {
+      const float f = exp2f((a.ref_d - a.md) * kLog2e);
       a.s1d = make_float2(f * a.s1d.x, f * a.s1d.y);
       a.skd = make_float2(f * a.skd.x, f * a.skd.y);
     }
-    a.md = m;
-    a.ad = v;
+    a.ref_d = a.md;
   }
-  const float y = fmaf(l, kLog2e, -a.mt * kLog2e);
+  const float y = fmaf(l, kLog2e, -a.ref_t * kLog2e);
   const float et = fast_exp2(y);
   a.s1t.x += et;
   a.s2t.x = fmaf(et, y, a.s2t.x);
-  const float ed = fast_exp2(fmaf(m, kLog2e, -a.md * kLog2e));
+  const float ed = fast_exp2(fmaf(m, kLog2e, -a.ref_d * kLog2e));
   a.s1d.x += ed;
   a.skd.x = fmaf(ed, m - l, a.skd.x);
   if constexpr (SAMPLE) {
     const float st = fmaf(l, invT, g), sd = fmaf(m, invT, g);
-    if (st > a.bt) { a.bt = st; a.it = v; a.lt_at = l; }
-    if (sd > a.bd) { a.bd = sd; a.id = v; }
+    if (st > a.bt) { a.bt = st; a.vbt = -1 - v; }
+    if (sd > a.bd) { a.bd = sd; a.vbd = -1 - v; }
   }
+}
+
+// Turn a thread's state for one row piece into a Partial: sums re-expressed
+// relative to the exact maximum, exact indices recovered by re-reading the one
+// 16-byte vector where each maximum / best score first appeared.
+template <typename T, bool SAMPLE>
+__device__ Partial resolve(const Acc& a, const T* lrow, const T* mrow, int pos, int b,
+                           const NoiseKey& key, float invT) {
+  constexpr int VEC = Unpack<T>::N;
+  Partial p;
+  p.mt = a.mt;
+  p.md = a.md;
+  p.s1t = p.s2t = p.s1d = p.skd = 0.f;
+  p.at = p.ad = p.it = p.id = 0x7fffffff;
+  p.bt = a.bt;
+  p.bd = a.bd;
+  p.lt_at = 0.f;
+  if (a.mt != -INFINITY) {
+    const float dl = (a.ref_t - a.mt) * kLog2e;  // <= 0
+    const float f = exp2f(dl);
+    const float s1 = a.s1t.x + a.s1t.y, s2 = a.s2t.x + a.s2t.y;
+    p.s1t = f * s1;
+    p.s2t = f * (s2 + dl * s1);
+    if (a.vt < 0) {
+      p.at = -1 - a.vt;
+    } else {
+      float x[VEC];
+      Vec<T>::unpack(*reinterpret_cast<const uint4*>(lrow + a.vt), x);
+      for (int e = VEC - 1; e >= 0; --e)
+        if (x[e] == a.mt) p.at = a.vt + e;
+    }
+  }
+  if (a.md != -INFINITY) {
+    const float f = exp2f((a.ref_d - a.md) * kLog2e);
+    p.s1d = f * (a.s1d.x + a.s1d.y);
+    p.skd = f * (a.skd.x + a.skd.y);
+    if (a.vd < 0) {
+      p.ad = -1 - a.vd;
+    } else {
+      float x[VEC];
+      Vec<T>::unpack(*reinterpret_cast<const uint4*>(mrow + a.vd), x);
+      for (int e = VEC - 1; e >= 0; --e)
+        if (x[e] == a.md) p.ad = a.vd + e;
+    }
+  }
+  if constexpr (SAMPLE) {
+    auto find = [&](int vb, float best, const T* row, int& idx, float* lval) {
+      if (best == -INFINITY) return;
+      if (vb < 0) {
+        idx = -1 - vb;
+        if (lval) *lval = Vec<T>::scalar(lrow + idx);
+        return;
+      }
+      float x[VEC], l[VEC], g[VEC];
+      Vec<T>::unpack(*reinterpret_cast<const uint4*>(row + vb), x);
+      Vec<T>::unpack(*reinterpret_cast<const uint4*>(lrow + vb), l);
+      for (int q = 0; q < VEC / 4; ++q) {
+        const PhiloxOut o = philox4x32_10((uint32_t)(vb >> 2) + q, (uint32_t)pos, (uint32_t)b,
+                                          key.step, key.k0, key.k1);
+        for (int w = 0; w < 4; ++w) g[4 * q + w] = gumbel_from_word(o.w[w]);
+      }
+      for (int e = VEC - 1; e >= 0; --e)
+        if (fmaf(x[e], invT, g[e]) == best) {
+          idx = vb + e;
+          if (lval) *lval = l[e];
+        }
+    };
+    find(a.vbt, a.bt, lrow, p.it, &p.lt_at);
+    find(a.vbd, a.bd, mrow, p.id, nullptr);
+  }
+  return p;
 }
 
 // Merge partial b into a (both cover disjoint vocabulary ranges of one row).
@@ -357,27 +397,6 @@ __device__ __forceinline__ Partial shfl_xor(const Partial& p, int mask) {
   q.id = __shfl_xor_sync(0xffffffffu, p.id, mask);
   return q;
 }
-
-template <typename T>
-struct Vec;
-template <>
-struct Vec<__nv_bfloat16> {
-  static constexpr int N = 8;
-  __device__ static void unpack(const uint4& u, float (&x)[8]) {
-    x[0] = bf16lo(u.x); x[1] = bf16hi(u.x); x[2] = bf16lo(u.y); x[3] = bf16hi(u.y);
-    x[4] = bf16lo(u.z); x[5] = bf16hi(u.z); x[6] = bf16lo(u.w); x[7] = bf16hi(u.w);
-  }
-  __device__ static float scalar(const __nv_bfloat16* p) { return __bfloat162float(*p); }
-};
-template <>
-struct Vec<float> {
-  static constexpr int N = 4;
-  __device__ static void unpack(const uint4& u, float (&x)[4]) {
-    x[0] = __uint_as_float(u.x); x[1] = __uint_as_float(u.y);
-    x[2] = __uint_as_float(u.z); x[3] = __uint_as_float(u.w);
-  }
-  __device__ static float scalar(const float* p) { return *p; }
-};
 
 // Gumbel noise of N consecutive entries starting at v0 (v0 % 4 == 0 when N >= 4).
 template <int N>
@@ -453,8 +472,7 @@ verify_stream_kernel(const VerifyArgs a) {
 
   Acc acc;
   init(acc);
-  auto flush = [&](int64_t row) {
-    Partial p = to_partial(acc);
+  auto flush = [&](int64_t row, Partial p) {
 #pragma unroll
     for (int mask = 16; mask > 0; mask >>= 1) {
       const Partial q = shfl_xor(p, mask);
@@ -467,9 +485,9 @@ verify_stream_kernel(const VerifyArgs a) {
       if (lane < kVThreads / 32) {
         r = red[lane];
       } else {
-        Acc e;
-        init(e);
-        r = to_partial(e);
+        r = p;  // an empty partial (no entries)
+        r.mt = r.md = r.bt = r.bd = -INFINITY;
+        r.s1t = r.s2t = r.s1d = r.skd = 0.f;
       }
 #pragma unroll
       for (int mask = 16; mask > 0; mask >>= 1) {
@@ -542,7 +560,7 @@ verify_stream_kernel(const VerifyArgs a) {
                          Vec<T>::scalar(LM + row * a.ld + e), g, e, a.invT);
       }
     }
-    flush(row);
+    flush(row, resolve<T, SAMPLE>(acc, LT + row * a.ld, LM + row * a.ld, pos, b, a.key, a.invT));
     sidx += vend - vbeg;
   }
 }
