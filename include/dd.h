@@ -169,6 +169,35 @@ dd_status dd_verify_logits(
 size_t dd_verify_logits_workspace_size(int B, int R, int V, dd_dtype dtype);
 
 /*
+ * dd_verify_logits_static -- dd_verify_logits for callers that cannot allocate
+ * device memory. (The pages have no counterpart: this is a library convenience.)
+ *
+ * Some callers cannot call cudaMalloc or supply a workspace: code embedded in a
+ * runtime that owns and budgets all device memory, latency-critical loops where
+ * an allocation's implicit device synchronisation is unacceptable, or code that
+ * must not hit out-of-memory mid-step. This entry point allocates nothing: the
+ * per-row partial states live in a fixed array of DD_STATIC_SCRATCH_BYTES inside
+ * libdd's own device memory, which every GPU that loads the library holds until
+ * the process exits. Same arguments, semantics and outputs as dd_verify_logits,
+ * without the workspace.
+ *   - The first call on a device looks up that array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - Every call shares the one array and leaves its contents behind; nothing in
+ *     it needs to start at zero. Calls that overlap on the GPU (e.g. on two
+ *     streams, or two threads) race on it: serialise them.
+ * Errors: as dd_verify_logits; DD_ERR_UNSUPPORTED when the call would need more
+ * than DD_STATIC_SCRATCH_BYTES of scratch (dd_verify_logits_workspace_size(...)
+ * > DD_STATIC_SCRATCH_BYTES) -- use dd_verify_logits with a workspace then;
+ * DD_ERR_CUDA if the array's address cannot be obtained.
+ */
+#define DD_STATIC_SCRATCH_BYTES (4u << 20)
+dd_status dd_verify_logits_static(
+    const void* logits_t, const void* logits_d, dd_dtype dtype,
+    int B, int R, int V, int64_t ld, int pos_offset,
+    float temperature, uint64_t seed, uint64_t step,
+    const dd_row_stats* out, void* stream);
+
+/*
  * dd_coupled_gumbel -- write the shared Gumbel noise g[b, r, v] (fp32, row
  * stride ld) that dd_verify_logits uses for row r = position pos_offset + r,
  * so that a drafter can sample with the very same noise ([SPOT] Coupled-Noise

@@ -5,3 +5,4 @@
 #include "dd_attention.cu"
 #include "dd_attention_tc.cu"
 #include "dd_select.cu"
+#include "dd_static.cu"

@@ -25,7 +25,7 @@ DD_MASK_TOKEN = -1
 # Every symbol include/dd.h declares.
 EXPORTED = (
     "dd_dualview_attention", "dd_dualview_attention_workspace_size", "dd_verify_logits",
-    "dd_verify_logits_workspace_size",
+    "dd_verify_logits_workspace_size", "dd_verify_logits_static",
     "dd_coupled_gumbel", "dd_select_seeds", "dd_decide", "dd_status_string",
     "dd_get_device_error", "dd_set_spin_limit", "dd_selftest_bounded_wait",
 )
@@ -69,6 +69,9 @@ def lib():
     L.dd_verify_logits.argtypes = [P, P, I, I, I, I, I64, I, F, U64, U64,
                                    ctypes.POINTER(_RowStats), P, SZ, P]
     L.dd_verify_logits.restype = I
+    L.dd_verify_logits_static.argtypes = [P, P, I, I, I, I, I64, I, F, U64, U64,
+                                          ctypes.POINTER(_RowStats), P]
+    L.dd_verify_logits_static.restype = I
     L.dd_verify_logits_workspace_size.argtypes = [I, I, I, I]
     L.dd_verify_logits_workspace_size.restype = SZ
     L.dd_coupled_gumbel.argtypes = [U64, U64, I, I, I, I64, I, P, P]
@@ -201,6 +204,25 @@ def dd_verify_logits(logits_t, logits_d, out: RowStats, pos_offset=0, temperatur
         int(seed) & (2**64 - 1), int(step) & (2**64 - 1), ctypes.byref(out._c()),
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
     _check("dd_verify_logits", st)
+
+
+def dd_verify_logits_static(logits_t, logits_d, out: RowStats, pos_offset=0, temperature=0.0,
+                            seed=0, step=0, stream=None):
+    """dd_verify_logits without a workspace: for callers that cannot allocate device
+    memory, the partial states live in a fixed array inside libdd (see include/dd.h for
+    its size limit and for why concurrent calls must not overlap)."""
+    B, R, V = logits_t.shape
+    if logits_t.stride(2) != 1 or logits_t.stride(0) != R * logits_t.stride(1):
+        raise ValueError("logits must be [B,R,V] with unit vocabulary stride and packed rows")
+    if logits_d.shape != logits_t.shape or logits_d.stride() != logits_t.stride():
+        raise ValueError("verifier and drafter logits must have the same shape and strides")
+    if not (logits_t.is_cuda and logits_d.is_cuda):
+        raise ValueError("libdd takes device memory: logits are on the CPU")
+    st = lib().dd_verify_logits_static(
+        ctypes.c_void_p(logits_t.data_ptr()), ctypes.c_void_p(logits_d.data_ptr()),
+        _dtype_code(logits_t), B, R, V, logits_t.stride(1), int(pos_offset), float(temperature),
+        int(seed) & (2**64 - 1), int(step) & (2**64 - 1), ctypes.byref(out._c()), _stream(stream))
+    _check("dd_verify_logits_static", st)
 
 
 def dd_coupled_gumbel(g, seed=0, step=0, pos_offset=0, stream=None):
