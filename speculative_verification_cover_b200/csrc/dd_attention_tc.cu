@@ -42,8 +42,7 @@ struct P1Layout {
   static constexpr int kQ = 0;
   static constexpr int kK = kQ + kTile;
   static constexpr int kV = kK + kStages * kTile;
-  static constexpr int kP = kV + kStages * kTile;
-  static constexpr int kB2 = kP + 2 * kAtom;          // P: 128 rows x 128 columns bf16
+  static constexpr int kB2 = kV + kStages * kTile;
   static constexpr int kB2Bytes = 2 * 16 * 128;       // 16 rows x 128 columns bf16
   // staging for up to kStaged seed rows of the step t-1 cache per stage (K then V rows)
   static constexpr int kStaged = 16;
@@ -61,11 +60,10 @@ struct P1Layout {
 
 struct P1Bars {
   uint64_t q_full;
-  uint64_t kv_full[kStages];
-  uint64_t kv_ready[kStages];
-  uint64_t kv_empty[kStages];
+  uint64_t k_full[kStages], k_ready[kStages], k_empty[kStages];
+  uint64_t v_full[kStages], v_ready[kStages], v_empty[kStages];
   uint64_t s_full[2];
-  uint64_t p_full;
+  uint64_t p_full[2];
   uint64_t pv_done;
   uint64_t drain;
   uint32_t tmem_base;
@@ -110,13 +108,17 @@ attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&bars->kv_full[s], 1);
-      mbar_init(&bars->kv_ready[s], 1);
-      mbar_init(&bars->kv_empty[s], 1);
+      mbar_init(&bars->k_full[s], 1);
+      mbar_init(&bars->k_ready[s], 1);
+      mbar_init(&bars->k_empty[s], 1);
+      mbar_init(&bars->v_full[s], 1);
+      mbar_init(&bars->v_ready[s], 1);
+      mbar_init(&bars->v_empty[s], 1);
     }
     mbar_init(&bars->s_full[0], 1);
     mbar_init(&bars->s_full[1], 1);
-    mbar_init(&bars->p_full, 4);
+    mbar_init(&bars->p_full[0], 4);
+    mbar_init(&bars->p_full[1], 4);
     mbar_init(&bars->pv_done, 1);
     mbar_init(&bars->drain, 1);
     bars->abort_flag = 0;
@@ -161,26 +163,31 @@ attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       neww[w] = p.newbits[(int64_t)b * W + w];
     }
     __syncwarp();
-    // Tile j: K/V from the current input, plus (same barrier) up to kStaged
-    // seed rows of the step t-1 cache into the stage's staging area.
-    auto issue = [&](int j) {
+    // Tile j of K (resp. V): the current input's rows, plus (same barrier) up to
+    // kStaged seed rows of the step t-1 cache into the stage's staging area. K
+    // and V have their own stages so K(j+2) can load as soon as QK(j) is done.
+    auto seeds_in_tile = [&](int j) {
+      int n = 0;
+      for (int w = 0; w < 4; ++w) {
+        const int wi = j * 4 + w;
+        n += wi < W ? __popc(seedw[wi]) : 0;
+      }
+      return min(n, Lay::kStaged);
+    };
+    auto issue = [&](int j, bool is_v) {
       const int s = j % kStages;
       if (lane == 0) {
-        int n = 0;
-        for (int w = 0; w < 4; ++w) {
-          const int wi = j * 4 + w;
-          n += wi < W ? __popc(seedw[wi]) : 0;
-        }
-        n = min(n, Lay::kStaged);
-        mbar_expect_tx(&bars->kv_full[s], kTxKV + 2u * n * Lay::kRowBytes);
+        const int n = seeds_in_tile(j);
+        uint64_t* bar = is_v ? &bars->v_full[s] : &bars->k_full[s];
+        mbar_expect_tx(bar, Lay::kTile + (uint32_t)n * Lay::kRowBytes);
+        const CUtensorMap* tm = is_v ? &tmV : &tmK;
+        const CUtensorMap* tmp = is_v ? &tmVp : &tmKp;
+        uint8_t* tile = smem + (is_v ? Lay::kV : Lay::kK) + s * Lay::kTile;
 #pragma unroll
-        for (int ac = 0; ac < D / 64; ++ac) {
-          tma_load_4d(smem + Lay::kK + s * Lay::kTile + ac * kAtom, &tmK, ac * 64, g, j * kBN, b,
-                      &bars->kv_full[s]);
-          tma_load_4d(smem + Lay::kV + s * Lay::kTile + ac * kAtom, &tmV, ac * 64, g, j * kBN, b,
-                      &bars->kv_full[s]);
-        }
-        uint8_t* stg = smem + Lay::kStage + s * Lay::kStageBytes;
+        for (int ac = 0; ac < D / 64; ++ac)
+          tma_load_4d(tile + ac * kAtom, tm, ac * 64, g, j * kBN, b, bar);
+        uint8_t* stg = smem + Lay::kStage + s * Lay::kStageBytes +
+                       (is_v ? Lay::kStaged * Lay::kRowBytes : 0);
         int slot = 0;
         for (int w = 0; w < 4 && slot < n; ++w) {
           const int wi = j * 4 + w;
@@ -188,51 +195,53 @@ attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           while (bits && slot < n) {
             const int r = w * 32 + __ffs(bits) - 1;
             bits &= bits - 1;
-            tma_load_4d(stg + slot * Lay::kRowBytes, &tmKp, 0, g, j * kBN + r, b,
-                        &bars->kv_full[s]);
-            tma_load_4d(stg + (Lay::kStaged + slot) * Lay::kRowBytes, &tmVp, 0, g, j * kBN + r,
-                        b, &bars->kv_full[s]);
+            tma_load_4d(stg + slot * Lay::kRowBytes, tmp, 0, g, j * kBN + r, b, bar);
             ++slot;
           }
         }
       }
     };
-    auto finalize = [&](int j) -> bool {
+    auto finalize = [&](int j, bool is_v) -> bool {
       const int s = j % kStages;
-      if (!wait_bounded(&bars->kv_full[s], (j / kStages) & 1, p.spin, abort_flag)) return false;
+      uint64_t* full = is_v ? &bars->v_full[s] : &bars->k_full[s];
+      if (!wait_bounded(full, (j / kStages) & 1, p.spin, abort_flag)) return false;
       const int col0 = j * kBN;
-      const uint32_t stg = sbase + Lay::kStage + s * Lay::kStageBytes;
-      const bool is_v = lane >= 16;
-      const int ch = lane & 15;
-      // drafting view: seed columns read the step t-1 cache
+      const uint32_t stg = sbase + Lay::kStage + s * Lay::kStageBytes +
+                           (is_v ? Lay::kStaged * Lay::kRowBytes : 0);
+      const uint32_t tile = sbase + (is_v ? Lay::kV : Lay::kK) + s * Lay::kTile;
+      const __nv_bfloat16* prev = is_v ? p.v_prev : p.k_prev;
+      // two seed rows at a time: lanes 0-15 and 16-31
+      const int half = lane >> 4, ch = lane & 15;
       int slot = 0;
       for (int w = 0; w < 4; ++w) {
         const int wi = j * 4 + w;
         uint32_t bits = wi < W ? seedw[wi] : 0u;
         while (bits) {
-          const int r = w * 32 + __ffs(bits) - 1;
+          int r0 = w * 32 + __ffs(bits) - 1;
           bits &= bits - 1;
-          if (ch < D / 8) {
+          int r1 = -1;
+          if (bits) {
+            r1 = w * 32 + __ffs(bits) - 1;
+            bits &= bits - 1;
+          }
+          const int r = half ? r1 : r0;
+          const int sl = slot + half;
+          if (r >= 0 && ch < D / 8) {
             uint4 val;
-            if (slot < Lay::kStaged) {
-              const uint32_t src =
-                  stg + ((is_v ? Lay::kStaged : 0) + slot) * Lay::kRowBytes + ch * 16;
+            if (sl < Lay::kStaged) {
               asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                            : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
-                           : "r"(src));
+                           : "r"(stg + sl * Lay::kRowBytes + ch * 16));
             } else {
-              val = ldg16((is_v ? p.v_prev : p.k_prev) +
-                          (((int64_t)b * L + col0 + r) * p.Hkv + g) * D + ch * 8);
+              val = ldg16(prev + (((int64_t)b * L + col0 + r) * p.Hkv + g) * D + ch * 8);
             }
-            const uint32_t dst = sbase + (is_v ? Lay::kV : Lay::kK) + s * Lay::kTile +
-                                 (ch / 8) * kAtom + sw128(r, ch & 7);
-            st_shared_v4(dst, val.x, val.y, val.z, val.w);
+            st_shared_v4(tile + (ch / 8) * kAtom + sw128(r, ch & 7), val.x, val.y, val.z, val.w);
           }
-          ++slot;
+          slot += r1 >= 0 ? 2 : 1;
         }
       }
-      // row 1 of the statistics operand: the tile's newly-written flags
-      if (lane < 16) {
+      if (is_v && lane < 16) {
+        // row 1 of the statistics operand: the tile's newly-written flags
         const int wi = j * 4 + lane / 4;
         const uint32_t byte = ((wi < W ? neww[wi] : 0u) >> ((lane & 3) * 8)) & 0xFFu;
         uint32_t w4[4];
@@ -245,29 +254,51 @@ attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
       fence_proxy_async();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->kv_ready[s]);
+      if (lane == 0) mbar_arrive(is_v ? &bars->v_ready[s] : &bars->k_ready[s]);
       return true;
     };
-    int issued = 0, finalized = 0;
-    for (int j = 0; j < T && j < kStages; ++j) { issue(j); ++issued; }
-    bool ok = finalize(0);
-    if (ok) finalized = 1;
+    int issued_k = 0, issued_v = 0, fin_k = 0, fin_v = 0;
+    for (int j = 0; j < T && j < kStages; ++j) {
+      issue(j, false);
+      ++issued_k;
+      issue(j, true);
+      ++issued_v;
+    }
+    bool ok = finalize(0, false);
+    if (ok) fin_k = 1;
+    ok = ok && finalize(0, true);
+    if (ok) fin_v = 1;
     for (int j = 0; ok && j < T; ++j) {
       if (j + 1 < T) {
-        ok = finalize(j + 1);
-        if (!ok) break;
-        finalized = j + 2;
+        if (!(ok = finalize(j + 1, false))) break;
+        fin_k = j + 2;
       }
       if (j + kStages < T) {
-        ok = wait_bounded(&bars->kv_empty[j % kStages], (j / kStages) & 1, p.spin, abort_flag);
-        if (!ok) break;
-        issue(j + kStages);
-        ++issued;
+        // K stage of tile j is free once QK(j) is done
+        if (!(ok = wait_bounded(&bars->k_empty[j % kStages], (j / kStages) & 1, p.spin,
+                                abort_flag)))
+          break;
+        issue(j + kStages, false);
+        ++issued_k;
+      }
+      if (j + 1 < T) {
+        if (!(ok = finalize(j + 1, true))) break;
+        fin_v = j + 2;
+      }
+      if (j + kStages < T) {
+        // V stage of tile j is free once PV(j) is done
+        if (!(ok = wait_bounded(&bars->v_empty[j % kStages], (j / kStages) & 1, p.spin,
+                                abort_flag)))
+          break;
+        issue(j + kStages, true);
+        ++issued_v;
       }
     }
     // never leave with TMA writes in flight
-    for (int j = finalized; j < issued; ++j)
-      wait_bounded(&bars->kv_full[j % kStages], (j / kStages) & 1, p.spin, abort_flag);
+    for (int j = fin_k; j < issued_k; ++j)
+      wait_bounded(&bars->k_full[j % kStages], (j / kStages) & 1, p.spin, abort_flag);
+    for (int j = fin_v; j < issued_v; ++j)
+      wait_bounded(&bars->v_full[j % kStages], (j / kStages) & 1, p.spin, abort_flag);
     wait_bounded(&bars->q_full, 0, p.spin, abort_flag);
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
@@ -286,9 +317,10 @@ attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           mma_bf16(dS, desc_kmajor_sw128(sQ + off), desc_kmajor_sw128(sK + off), idS, kk > 0);
         }
         mma_commit(&bars->s_full[j & 1]);
+        mma_commit(&bars->k_empty[s]);
       };
       bool ok = wait_bounded(&bars->q_full, 0, p.spin, abort_flag);
-      ok = ok && wait_bounded(&bars->kv_ready[0], 0, p.spin, abort_flag);
+      ok = ok && wait_bounded(&bars->k_ready[0], 0, p.spin, abort_flag);
       if (ok) {
         fence_after_sync();
         qk(0);
@@ -296,28 +328,31 @@ attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       for (int j = 0; ok && j < T; ++j) {
         if (j + 1 < T) {
           const int s1 = (j + 1) % kStages;
-          ok = wait_bounded(&bars->kv_ready[s1], ((j + 1) / kStages) & 1, p.spin, abort_flag);
+          ok = wait_bounded(&bars->k_ready[s1], ((j + 1) / kStages) & 1, p.spin, abort_flag);
+          // S(j+1) overwrites the buffer that held P(j-1): PV(j-1) must be done
+          if (ok && j >= 1) ok = wait_bounded(&bars->pv_done, (j - 1) & 1, p.spin, abort_flag);
           if (!ok) break;
           fence_after_sync();
           qk(j + 1);
         }
-        ok = wait_bounded(&bars->p_full, j & 1, p.spin, abort_flag);
+        const int s = j % kStages;
+        ok = wait_bounded(&bars->p_full[j & 1], (j >> 1) & 1, p.spin, abort_flag) &&
+             wait_bounded(&bars->v_ready[s], (j / kStages) & 1, p.spin, abort_flag);
         if (!ok) break;
         fence_after_sync();
-        const int s = j % kStages;
-        const uint32_t sP = sbase + Lay::kP;
+        const uint32_t tP = tmem + ((j & 1) ? Lay::kS1 : Lay::kS0);  // P(j), bf16 pairs
         const uint32_t sV = sbase + Lay::kV + s * Lay::kTile;
         const uint32_t sB2 = sbase + Lay::kB2 + s * Lay::kB2Bytes;
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint64_t a = desc_kmajor_sw128(sP + (kk / 4) * kAtom + (kk % 4) * 32);
           const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
-          mma_bf16(tmem + Lay::kO, a, desc_mnmajor_sw128(sV + kk * 16 * 128, kAtom), idO, acc);
-          mma_bf16(tmem + Lay::kSt, a, desc_kmajor_sw128(sB2 + (kk / 4) * 2048 + (kk % 4) * 32),
-                   idSt, acc);
+          mma_bf16_ts(tmem + Lay::kO, tP + kk * 8, desc_mnmajor_sw128(sV + kk * 16 * 128, kAtom),
+                      idO, acc);
+          mma_bf16_ts(tmem + Lay::kSt, tP + kk * 8,
+                      desc_kmajor_sw128(sB2 + (kk / 4) * 2048 + (kk % 4) * 32), idSt, acc);
         }
         mma_commit(&bars->pv_done);
-        mma_commit(&bars->kv_empty[s]);
+        mma_commit(&bars->v_empty[s]);
       }
       // all issued tensor-core work done before TMEM is released
       mma_commit(&bars->drain);
@@ -335,7 +370,6 @@ attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const float c2 = p.scale_log2;
     float m = -INFINITY;
     bool ok = true;
-    const uint32_t sP = sbase + Lay::kP;
     for (int j = 0; j < T; ++j) {
       ok = wait_bounded(&bars->s_full[j & 1], (j >> 1) & 1, p.spin, abort_flag);
       if (!ok) break;
@@ -362,19 +396,25 @@ attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         for (int c = 0; c < kBN; ++c)
           if (c == r) s[c] = -INFINITY;
       }
-      float mx = -INFINITY;
+      // row maximum: eight independent chains, then a tree (short dependency chain)
+      float pm[8];
 #pragma unroll
-      for (int c = 0; c < kBN; ++c) mx = fmaxf(mx, s[c]);
+      for (int e = 0; e < 8; ++e) pm[e] = s[e];
+#pragma unroll
+      for (int c = 8; c < kBN; c += 8)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) pm[e] = fmaxf(pm[e], s[c + e]);
+      float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                       fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
       mx *= c2;
       const bool need = mx > m + 8.f;
       const float m_new = need ? mx : m;
-      if (j > 0) {
+      const bool resc = need && j > 0 && m != -INFINITY;
+      if (__any_sync(0xffffffffu, resc)) {
+        // O (and the statistics columns) may only be rescaled once PV(j-1) is done
         ok = wait_bounded(&bars->pv_done, (j - 1) & 1, p.spin, abort_flag);
         if (!ok) break;
         fence_after_sync();
-      }
-      const bool resc = need && j > 0 && m != -INFINITY;
-      if (__any_sync(0xffffffffu, resc)) {
         const float f = resc ? exp2f(m - m_new) : 1.f;
 #pragma unroll 1
         for (int q = 0; q < D / 32 + 1; ++q) {
@@ -389,23 +429,29 @@ attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
       m = m_new;
       const bool live = m != -INFINITY;
+      // P = exp2(S * scale * log2e - m) as bf16 pairs over the first 64 columns of
+      // this tile's S buffer (already read into registers): the A operand of PV.
+      const uint32_t scol = (j & 1) ? Lay::kS1 : Lay::kS0;
 #pragma unroll
-      for (int cc = 0; cc < kBN / 8; ++cc) {
-        uint32_t w[4];
+      for (int half = 0; half < 2; ++half) {
+        uint32_t w[32];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float a = live ? fast_exp2(fmaf(s[cc * 8 + 2 * e], c2, -m)) : 0.f;
-          const float bb = live ? fast_exp2(fmaf(s[cc * 8 + 2 * e + 1], c2, -m)) : 0.f;
+        for (int e = 0; e < 32; ++e) {
+          const int c = half * 64 + 2 * e;
+          const float a = live ? fast_exp2(fmaf(s[c], c2, -m)) : 0.f;
+          const float bb = live ? fast_exp2(fmaf(s[c + 1], c2, -m)) : 0.f;
           w[e] = pack_bf16(a, bb);
         }
-        st_shared_v4(sP + (cc / 8) * kAtom + sw128(r, cc & 7), w[0], w[1], w[2], w[3]);
+        tmem_st32u(tl + scol + half * 32, w);
       }
-      fence_proxy_async();
+      tmem_wait_st();
       fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->p_full);
+      if (lane == 0) mbar_arrive(&bars->p_full[j & 1]);
     }
-    if (ok) ok = wait_bounded(&bars->pv_done, (T - 1) & 1, p.spin, abort_flag);
+    // Warps may be a tile apart, so pv_done's parity cannot tell PV(T-1) from
+    // PV(T-3) here; drain completes once, after every tensor-core operation.
+    if (ok) ok = wait_bounded(&bars->drain, 0, p.spin, abort_flag);
     if (ok) {
       fence_after_sync();
       float o[D];
