@@ -65,7 +65,7 @@ extern "C" {
 
 size_t dd_dualview_attention_workspace_size(int B, int L, int Hq, int Hkv, int d) {
   if (B < 1 || L < 1 || Hq < 1 || Hkv < 1 || d < 1) return 0;
-  return attn_workspace_layout(B, L, Hq).total;
+  return attn_workspace_layout(B, L, Hq, Hkv, d).total;
 }
 
 dd_status dd_dualview_attention(const void* q, const void* k_cur, const void* v_cur,
@@ -86,7 +86,7 @@ dd_status dd_dualview_attention(const void* q, const void* k_cur, const void* v_
       (k_prev && !aligned16(k_prev)) || (v_prev && !aligned16(v_prev)))
     return DD_ERR_INVALID_ARG;
   if (dtype == DD_BF16 && L > kTcMaxL) return DD_ERR_UNSUPPORTED;
-  const AttnWorkspace ws = attn_workspace_layout(B, L, Hq);
+  const AttnWorkspace ws = attn_workspace_layout(B, L, Hq, Hkv, d);
   if (!workspace || workspace_bytes < ws.total) return DD_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return DD_ERR_INVALID_ARG;
   AttnArgs a{};
@@ -104,6 +104,12 @@ dd_status dd_dualview_attention(const void* q, const void* k_cur, const void* v_
   a.mcount = reinterpret_cast<int32_t*>(w + ws.mcount_off);
   a.seedbits = reinterpret_cast<uint32_t*>(w + ws.seedbits_off);
   a.newbits = reinterpret_cast<uint32_t*>(w + ws.newbits_off);
+  a.mrank = reinterpret_cast<int32_t*>(w + ws.mrank_off);
+  a.k_view = w + ws.kview_off;
+  a.v_view = w + ws.vview_off;
+  a.q_m = w + ws.qm_off;
+  a.lse2_m = reinterpret_cast<float*>(w + ws.lse2m_off);
+  a.Lp = ws.Lp;
   return from_cuda(launch_attention(a, static_cast<cudaStream_t>(stream)));
 }
 

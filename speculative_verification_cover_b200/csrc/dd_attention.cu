@@ -16,7 +16,7 @@
 
 namespace dd {
 
-AttnWorkspace attn_workspace_layout(int B, int L, int Hq) {
+AttnWorkspace attn_workspace_layout(int B, int L, int Hq, int Hkv, int d) {
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
   AttnWorkspace w;
   const size_t part = (size_t)B * Hq * L * sizeof(float);
@@ -27,35 +27,81 @@ AttnWorkspace attn_workspace_layout(int B, int L, int Hq) {
   const size_t words = (size_t)B * ((L + 31) / 32) * sizeof(uint32_t);
   w.seedbits_off = up(w.mcount_off + (size_t)B * sizeof(int32_t));
   w.newbits_off = up(w.seedbits_off + words);
-  w.total = up(w.newbits_off + words);
+  w.mrank_off = up(w.newbits_off + words);
+  // tensor-core path: bf16 views and the compacted masked rows for pass 2
+  w.Lp = (L + 127) / 128 * 128;
+  const size_t kv = (size_t)B * L * Hkv * d * 2;
+  w.kview_off = up(w.mrank_off + (size_t)B * L * sizeof(int32_t));
+  w.vview_off = up(w.kview_off + kv);
+  w.qm_off = up(w.vview_off + kv);
+  w.lse2m_off = up(w.qm_off + (size_t)B * L * Hq * d * 2);
+  w.total = up(w.lse2m_off + (size_t)B * Hq * w.Lp * sizeof(float));
   return w;
 }
 
 namespace {
 
 // ---------------------------------------------------------------------------
-// Per sequence: the masked query rows in ascending order (stable compaction),
-// and the seed / newly-written flags packed 32 to a word.
-__global__ void __launch_bounds__(1024) prep_kernel(const uint8_t* __restrict__ is_masked,
-                                                    const uint8_t* __restrict__ is_seed,
-                                                    const uint8_t* __restrict__ is_new, int L,
-                                                    int32_t* __restrict__ mrows,
-                                                    int32_t* __restrict__ mcount,
-                                                    uint32_t* __restrict__ seedbits,
-                                                    uint32_t* __restrict__ newbits) {
-  const int b = blockIdx.x;
+// Everything the passes need from the flags, one launch, grid (1 + copy blocks, B):
+//   block 0 of sequence b: the seed / newly-written flags packed 32 to a word, the
+//     masked query rows in ascending order (stable compaction), their count, and
+//     each row's rank among them (-1 for a row that is not masked);
+//   blocks 1.. (tensor-core path with seeds): the drafting view of K and V --
+//     row j of the step t-1 cache where j is a seed, of the current input
+//     otherwise -- so the attention passes stream plain tiles of it.
+struct PrepArgs {
+  const uint8_t *is_masked, *is_seed, *is_new;
+  int L;
+  int32_t *mrows, *mcount, *mrank;  // mrows == nullptr: no compaction
+  uint32_t *seedbits, *newbits;
+  // drafting view (view_units == 0: none); rows of row_units 16-byte units
+  const uint4 *k_cur, *v_cur, *k_prev, *v_prev;
+  uint4 *k_view, *v_view;
+  int64_t view_units;  // per sequence: L * row_units
+  int row_units;       // Hkv * d * 2 / 16
+};
+constexpr int kPrepThreads = 1024;
+constexpr int kPrepUnitsPerThread = 4;
+
+__global__ void __launch_bounds__(kPrepThreads) prep_kernel(const PrepArgs a) {
+  const int b = blockIdx.y;
+  const int L = a.L;
+  if (blockIdx.x > 0) {
+    const int64_t base = (int64_t)b * a.view_units;
+    const int64_t u0 = (int64_t)(blockIdx.x - 1) * (kPrepThreads * kPrepUnitsPerThread) + threadIdx.x;
+    uint4 kv[kPrepUnitsPerThread], vv[kPrepUnitsPerThread];
+#pragma unroll
+    for (int e = 0; e < kPrepUnitsPerThread; ++e) {
+      const int64_t u = u0 + e * kPrepThreads;
+      if (u < a.view_units) {
+        const int pos = (int)(u / a.row_units);
+        const bool seed = a.is_seed[(int64_t)b * L + pos] != 0;
+        kv[e] = (seed ? a.k_prev : a.k_cur)[base + u];
+        vv[e] = (seed ? a.v_prev : a.v_cur)[base + u];
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < kPrepUnitsPerThread; ++e) {
+      const int64_t u = u0 + e * kPrepThreads;
+      if (u < a.view_units) {
+        a.k_view[base + u] = kv[e];
+        a.v_view[base + u] = vv[e];
+      }
+    }
+    return;
+  }
   const int W = (L + 31) / 32;
   for (int i0 = threadIdx.x & ~31; i0 < W * 32; i0 += blockDim.x) {
     const int i = i0 + (threadIdx.x & 31);
-    const bool fs = is_seed != nullptr && i < L && is_seed[(int64_t)b * L + i];
-    const bool fn = is_new != nullptr && i < L && is_new[(int64_t)b * L + i];
+    const bool fs = a.is_seed != nullptr && i < L && a.is_seed[(int64_t)b * L + i];
+    const bool fn = a.is_new != nullptr && i < L && a.is_new[(int64_t)b * L + i];
     const uint32_t ws = __ballot_sync(0xffffffffu, fs), wn = __ballot_sync(0xffffffffu, fn);
     if ((threadIdx.x & 31) == 0) {
-      if (seedbits) seedbits[(int64_t)b * W + i0 / 32] = ws;
-      if (newbits) newbits[(int64_t)b * W + i0 / 32] = wn;
+      if (a.seedbits) a.seedbits[(int64_t)b * W + i0 / 32] = ws;
+      if (a.newbits) a.newbits[(int64_t)b * W + i0 / 32] = wn;
     }
   }
-  if (mrows == nullptr) return;
+  if (a.mrows == nullptr) return;
   __shared__ int warp_sums[32];
   __shared__ int base;
   if (threadIdx.x == 0) base = 0;
@@ -63,7 +109,7 @@ __global__ void __launch_bounds__(1024) prep_kernel(const uint8_t* __restrict__ 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
   for (int c0 = 0; c0 < L; c0 += blockDim.x) {
     const int i = c0 + threadIdx.x;
-    const int f = (is_masked != nullptr && i < L && is_masked[(int64_t)b * L + i]) ? 1 : 0;
+    const int f = (a.is_masked != nullptr && i < L && a.is_masked[(int64_t)b * L + i]) ? 1 : 0;
     int incl = f;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -74,7 +120,9 @@ __global__ void __launch_bounds__(1024) prep_kernel(const uint8_t* __restrict__ 
     __syncthreads();
     int before = 0;
     for (int w = 0; w < warp; ++w) before += warp_sums[w];
-    if (f) mrows[(int64_t)b * L + base + before + incl - 1] = i;
+    const int rank = base + before + incl - 1;
+    if (f) a.mrows[(int64_t)b * L + rank] = i;
+    if (i < L) a.mrank[(int64_t)b * L + i] = f ? rank : -1;
     __syncthreads();
     if (threadIdx.x == 0) {
       int tot = 0;
@@ -83,7 +131,7 @@ __global__ void __launch_bounds__(1024) prep_kernel(const uint8_t* __restrict__ 
     }
     __syncthreads();
   }
-  if (threadIdx.x == 0) mcount[b] = base;
+  if (threadIdx.x == 0) a.mcount[b] = base;
 }
 
 // d_x[b, j] = (accumulate ? d_x[b, j] : 0) + (1/Hq) sum_s part[b, s, j], s < nslices,
@@ -383,9 +431,31 @@ cudaError_t launch_attention_tc(const AttnArgs& a, cudaStream_t stream, bool* ha
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t stream) {
   cudaError_t err;
   const bool need_din = a.d_in != nullptr && a.is_masked != nullptr;
-  prep_kernel<<<a.B, 1024, 0, stream>>>(a.is_masked, a.is_seed, a.is_new, a.L,
-                                        need_din ? a.mrows : nullptr, a.mcount, a.seedbits,
-                                        a.newbits);
+  PrepArgs pa{};
+  pa.is_masked = a.is_masked;
+  pa.is_seed = a.is_seed;
+  pa.is_new = a.is_new;
+  pa.L = a.L;
+  pa.mrows = need_din ? a.mrows : nullptr;
+  pa.mcount = a.mcount;
+  pa.mrank = a.mrank;
+  pa.seedbits = a.seedbits;
+  pa.newbits = a.newbits;
+  unsigned copy_blocks = 0;
+  if (a.dtype == DD_BF16 && a.is_seed != nullptr) {
+    // the tensor-core passes read the drafting view instead of patching tiles
+    pa.k_cur = static_cast<const uint4*>(a.k_cur);
+    pa.v_cur = static_cast<const uint4*>(a.v_cur);
+    pa.k_prev = static_cast<const uint4*>(a.k_prev);
+    pa.v_prev = static_cast<const uint4*>(a.v_prev);
+    pa.k_view = static_cast<uint4*>(a.k_view);
+    pa.v_view = static_cast<uint4*>(a.v_view);
+    pa.row_units = a.Hkv * a.d * 2 / 16;
+    pa.view_units = (int64_t)a.L * pa.row_units;
+    const int64_t per_block = kPrepThreads * kPrepUnitsPerThread;
+    copy_blocks = (unsigned)((pa.view_units + per_block - 1) / per_block);
+  }
+  prep_kernel<<<dim3(1 + copy_blocks, a.B), kPrepThreads, 0, stream>>>(pa);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   bool handled = false;
   int din_slices = a.Hq;  // d_in partials: per query head (CUDA-core pass 2) or per kv head

@@ -1,22 +1,27 @@
 // Tensor-core (sm_100a, tcgen05) dual-view attention for bf16 inputs.
 //
+// The drafting view -- seed rows of K and V taken from the step t-1 cache --
+// is materialised once per call by the prep kernel, so both passes stream
+// plain TMA tiles of it and no tile is patched on the way in.
+//
 // Pass 1, one CTA per (128 query rows, head, sequence), warp-specialised:
-//   warp 0      producer: TMA loads of the Q tile and of K/V tiles (128 columns,
-//               two stages) from k_cur / v_cur; then, per tile, overwrites the
-//               rows of seed columns with the step t-1 cache (k_prev / v_prev,
-//               plain loads + swizzled shared stores) -- the drafting view; and
-//               writes the tile's "newly written" flags into a small B operand
-//               whose rows are [1, is_new, 0, ...].
+//   warp 0      producer: TMA loads of the Q tile and of K / V tiles of the
+//               view (128 columns; K and V have their own stage rings), and the
+//               tile's "newly written" flags as row 1 of a small B operand whose
+//               rows are [1, is_new, 0, ...].
 //   warp 1      MMA issuer (one thread): S = Q K^T into a double-buffered TMEM
-//               accumulator; O += P V and [l, l_new] += P [1, is_new]^T, i.e. the
-//               row sum and the mass on newly written columns come out of the
-//               tensor core with the same bf16 P that weights V.
+//               accumulator; O += P V and [l, l_new] += P [1, is_new]^T with P
+//               read from TMEM, i.e. the row sum and the mass on newly written
+//               columns come out of the tensor core with the same bf16 P that
+//               weights V.
 //   warps 2-5   softmax (one thread per query row = TMEM lane): online max with
 //               a lazy rescale (O is rescaled in TMEM only when the running max
-//               grows by more than 2^8), P = exp2(S*scale*log2e - m) as bf16 into
-//               shared memory. A seed query's own column is masked in the loop and
-//               merged back afterwards from k_cur / v_cur (leave-one-out
-//               diagonal). Epilogue: out = O / l, lse, d_out partial = l_new / l.
+//               grows by more than 2^8), P = exp2(S*scale*log2e - m) as bf16
+//               pairs written over the S columns they came from. A seed query's
+//               own column is masked in the loop and merged back afterwards from
+//               k_cur / v_cur (leave-one-out diagonal). Epilogue: out = O / l,
+//               lse, d_out partial = l_new / l, and for a still-masked row its Q
+//               row and lse (log2 units) in rank order, the inputs of pass 2.
 // Every wait is bounded; on expiry the kernel records DD_ERR_TIMEOUT and winds down.
 #include <cudaTypedefs.h>
 
@@ -31,7 +36,8 @@ using namespace tc;
 
 constexpr int kBM = 128;
 constexpr int kBN = 128;
-constexpr int kStages = 2;
+constexpr int kSK = 3;  // K stages
+constexpr int kSV = 2;  // V stages
 constexpr int kP1Threads = 192;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kAtom = 128 * 128;  // one 128-row x 128-byte swizzle atom column
@@ -41,18 +47,13 @@ struct P1Layout {
   static constexpr int kTile = (D / 64) * kAtom;  // 128 x D bf16
   static constexpr int kQ = 0;
   static constexpr int kK = kQ + kTile;
-  static constexpr int kV = kK + kStages * kTile;
-  static constexpr int kB2 = kV + kStages * kTile;
-  static constexpr int kB2Bytes = 2 * 16 * 128;       // 16 rows x 128 columns bf16
-  // staging for up to kStaged seed rows of the step t-1 cache per stage (K then V rows)
-  static constexpr int kStaged = 16;
-  static constexpr int kRowBytes = D * 2;
-  static constexpr int kStage = kB2 + kStages * kB2Bytes;
-  static constexpr int kStageBytes = 2 * kStaged * kRowBytes;
-  // packed seed / newly-written flags of the whole sequence
-  static constexpr int kMask = kStage + kStages * kStageBytes;
-  static constexpr int kMaskWords = kTcMaxL / 32;
-  static constexpr int kBar = kMask + 2 * kMaskWords * 4;
+  static constexpr int kV = kK + kSK * kTile;
+  static constexpr int kB2 = kV + kSV * kTile;
+  static constexpr int kB2Bytes = 2 * 16 * 128;  // 16 rows x 128 columns bf16
+  // packed newly-written flags of the whole sequence
+  static constexpr int kNew = kB2 + kSV * kB2Bytes;
+  static constexpr int kNewWords = kTcMaxL / 32;
+  static constexpr int kBar = kNew + kNewWords * 4;
   static constexpr int kBytes = kBar + 256;
   // TMEM columns
   static constexpr uint32_t kS0 = 0, kS1 = 128, kO = 256, kSt = 256 + D;
@@ -60,8 +61,8 @@ struct P1Layout {
 
 struct P1Bars {
   uint64_t q_full;
-  uint64_t k_full[kStages], k_ready[kStages], k_empty[kStages];
-  uint64_t v_full[kStages], v_ready[kStages], v_empty[kStages];
+  uint64_t k_full[kSK], k_empty[kSK];
+  uint64_t v_full[kSV], v_empty[kSV];
   uint64_t s_full[2];
   uint64_t p_full[2];
   uint64_t pv_done;
@@ -71,14 +72,17 @@ struct P1Bars {
 };
 
 struct P1Params {
-  const __nv_bfloat16 *q, *k_cur, *v_cur, *k_prev, *v_prev;
+  const __nv_bfloat16 *q, *k_cur, *v_cur;
   const uint8_t *is_seed, *is_new;
-  const uint32_t *seedbits, *newbits;  // [B, ceil(L/32)]
-  int L, Hq, Hkv;
+  const uint32_t* newbits;  // [B, ceil(L/32)]
+  const int32_t* mrank;     // [B, L]
+  int L, Hq, Hkv, Lp;
   float scale_log2;
   __nv_bfloat16* out;
   float* lse;
   float* dout_part;
+  __nv_bfloat16* q_m;  // nullptr: pass 2 does not run
+  float* lse2_m;
   uint32_t spin;
 };
 
@@ -89,8 +93,7 @@ __device__ __forceinline__ uint4 ldg16(const void* p) {
 template <int D>
 __global__ void __launch_bounds__(kP1Threads, 1)
 attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKp,
-               const __grid_constant__ CUtensorMap tmVp, const P1Params p) {
+               const __grid_constant__ CUtensorMap tmV, const P1Params p) {
   using Lay = P1Layout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -107,12 +110,12 @@ attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kSK; ++s) {
       mbar_init(&bars->k_full[s], 1);
-      mbar_init(&bars->k_ready[s], 1);
       mbar_init(&bars->k_empty[s], 1);
+    }
+    for (int s = 0; s < kSV; ++s) {
       mbar_init(&bars->v_full[s], 1);
-      mbar_init(&bars->v_ready[s], 1);
       mbar_init(&bars->v_empty[s], 1);
     }
     mbar_init(&bars->s_full[0], 1);
@@ -131,7 +134,7 @@ attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   // constant rows of the [1, is_new, 0...] operand: row 0 = ones, rows 2..15 = 0
   if (warp >= 2) {
     const int t = threadIdx.x - 64;  // 0..127
-    for (int idx = t; idx < kStages * 2 * 16 * 8; idx += 128) {
+    for (int idx = t; idx < kSV * 2 * 16 * 8; idx += 128) {
       const int s = idx / (2 * 16 * 8), rem = idx % (2 * 16 * 8);
       const int ac = rem / (16 * 8), row = (rem / 8) % 16, c = rem % 8;
       const uint32_t one = 0x3F803F80u;  // two bf16 1.0
@@ -147,100 +150,35 @@ attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
   if (warp == 0) {
     // ------------------------------------------------------------------ producer
-    constexpr uint32_t kTxQ = Lay::kTile, kTxKV = 2 * Lay::kTile;
     if (lane == 0) {
-      mbar_expect_tx(&bars->q_full, kTxQ);
+      mbar_expect_tx(&bars->q_full, Lay::kTile);
 #pragma unroll
       for (int ac = 0; ac < D / 64; ++ac)
         tma_load_4d(smem + Lay::kQ + ac * kAtom, &tmQ, ac * 64, h, q0, b, &bars->q_full);
     }
-    // the sequence's packed flags into shared memory
-    uint32_t* seedw = reinterpret_cast<uint32_t*>(smem + Lay::kMask);
-    uint32_t* neww = seedw + Lay::kMaskWords;
+    uint32_t* neww = reinterpret_cast<uint32_t*>(smem + Lay::kNew);
     const int W = (L + 31) / 32;
-    for (int w = lane; w < W; w += 32) {
-      seedw[w] = p.seedbits[(int64_t)b * W + w];
-      neww[w] = p.newbits[(int64_t)b * W + w];
-    }
+    for (int w = lane; w < W; w += 32) neww[w] = p.newbits[(int64_t)b * W + w];
     __syncwarp();
-    // Tile j of K (resp. V): the current input's rows, plus (same barrier) up to
-    // kStaged seed rows of the step t-1 cache into the stage's staging area. K
-    // and V have their own stages so K(j+2) can load as soon as QK(j) is done.
-    auto seeds_in_tile = [&](int j) {
-      int n = 0;
-      for (int w = 0; w < 4; ++w) {
-        const int wi = j * 4 + w;
-        n += wi < W ? __popc(seedw[wi]) : 0;
-      }
-      return min(n, Lay::kStaged);
-    };
-    auto issue = [&](int j, bool is_v) {
-      const int s = j % kStages;
+    // K(j) may reuse its stage once QK(j - kSK) is done, V(j) once PV(j - kSV) is.
+    auto issue_k = [&](int j) -> bool {
+      const int s = j % kSK;
+      if (j >= kSK && !wait_bounded(&bars->k_empty[s], ((j / kSK) - 1) & 1, p.spin, abort_flag))
+        return false;
       if (lane == 0) {
-        const int n = seeds_in_tile(j);
-        uint64_t* bar = is_v ? &bars->v_full[s] : &bars->k_full[s];
-        mbar_expect_tx(bar, Lay::kTile + (uint32_t)n * Lay::kRowBytes);
-        const CUtensorMap* tm = is_v ? &tmV : &tmK;
-        const CUtensorMap* tmp = is_v ? &tmVp : &tmKp;
-        uint8_t* tile = smem + (is_v ? Lay::kV : Lay::kK) + s * Lay::kTile;
+        mbar_expect_tx(&bars->k_full[s], Lay::kTile);
 #pragma unroll
         for (int ac = 0; ac < D / 64; ++ac)
-          tma_load_4d(tile + ac * kAtom, tm, ac * 64, g, j * kBN, b, bar);
-        uint8_t* stg = smem + Lay::kStage + s * Lay::kStageBytes +
-                       (is_v ? Lay::kStaged * Lay::kRowBytes : 0);
-        int slot = 0;
-        for (int w = 0; w < 4 && slot < n; ++w) {
-          const int wi = j * 4 + w;
-          uint32_t bits = wi < W ? seedw[wi] : 0u;
-          while (bits && slot < n) {
-            const int r = w * 32 + __ffs(bits) - 1;
-            bits &= bits - 1;
-            tma_load_4d(stg + slot * Lay::kRowBytes, tmp, 0, g, j * kBN + r, b, bar);
-            ++slot;
-          }
-        }
+          tma_load_4d(smem + Lay::kK + s * Lay::kTile + ac * kAtom, &tmK, ac * 64, g, j * kBN, b,
+                      &bars->k_full[s]);
       }
+      return true;
     };
-    auto finalize = [&](int j, bool is_v) -> bool {
-      const int s = j % kStages;
-      uint64_t* full = is_v ? &bars->v_full[s] : &bars->k_full[s];
-      if (!wait_bounded(full, (j / kStages) & 1, p.spin, abort_flag)) return false;
-      const int col0 = j * kBN;
-      const uint32_t stg = sbase + Lay::kStage + s * Lay::kStageBytes +
-                           (is_v ? Lay::kStaged * Lay::kRowBytes : 0);
-      const uint32_t tile = sbase + (is_v ? Lay::kV : Lay::kK) + s * Lay::kTile;
-      const __nv_bfloat16* prev = is_v ? p.v_prev : p.k_prev;
-      // two seed rows at a time: lanes 0-15 and 16-31
-      const int half = lane >> 4, ch = lane & 15;
-      int slot = 0;
-      for (int w = 0; w < 4; ++w) {
-        const int wi = j * 4 + w;
-        uint32_t bits = wi < W ? seedw[wi] : 0u;
-        while (bits) {
-          int r0 = w * 32 + __ffs(bits) - 1;
-          bits &= bits - 1;
-          int r1 = -1;
-          if (bits) {
-            r1 = w * 32 + __ffs(bits) - 1;
-            bits &= bits - 1;
-          }
-          const int r = half ? r1 : r0;
-          const int sl = slot + half;
-          if (r >= 0 && ch < D / 8) {
-            uint4 val;
-            if (sl < Lay::kStaged) {
-              asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                           : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
-                           : "r"(stg + sl * Lay::kRowBytes + ch * 16));
-            } else {
-              val = ldg16(prev + (((int64_t)b * L + col0 + r) * p.Hkv + g) * D + ch * 8);
-            }
-            st_shared_v4(tile + (ch / 8) * kAtom + sw128(r, ch & 7), val.x, val.y, val.z, val.w);
-          }
-          slot += r1 >= 0 ? 2 : 1;
-        }
-      }
-      if (is_v && lane < 16) {
+    auto issue_v = [&](int j) -> bool {
+      const int s = j % kSV;
+      if (j >= kSV && !wait_bounded(&bars->v_empty[s], ((j / kSV) - 1) & 1, p.spin, abort_flag))
+        return false;
+      if (lane < 16) {
         // row 1 of the statistics operand: the tile's newly-written flags
         const int wi = j * 4 + lane / 4;
         const uint32_t byte = ((wi < W ? neww[wi] : 0u) >> ((lane & 3) * 8)) & 0xFFu;
@@ -254,51 +192,36 @@ attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
       fence_proxy_async();
       __syncwarp();
-      if (lane == 0) mbar_arrive(is_v ? &bars->v_ready[s] : &bars->k_ready[s]);
+      if (lane == 0) {
+        mbar_expect_tx(&bars->v_full[s], Lay::kTile);
+#pragma unroll
+        for (int ac = 0; ac < D / 64; ++ac)
+          tma_load_4d(smem + Lay::kV + s * Lay::kTile + ac * kAtom, &tmV, ac * 64, g, j * kBN, b,
+                      &bars->v_full[s]);
+      }
       return true;
     };
-    int issued_k = 0, issued_v = 0, fin_k = 0, fin_v = 0;
-    for (int j = 0; j < T && j < kStages; ++j) {
-      issue(j, false);
-      ++issued_k;
-      issue(j, true);
-      ++issued_v;
-    }
-    bool ok = finalize(0, false);
-    if (ok) fin_k = 1;
-    ok = ok && finalize(0, true);
-    if (ok) fin_v = 1;
+    // the order the MMA issuer consumes them: K0, K1, V0, K2, V1, K3, V2, ...
+    int nk = 0, nv = 0;
+    bool ok = issue_k(0);
+    if (ok) nk = 1;
     for (int j = 0; ok && j < T; ++j) {
       if (j + 1 < T) {
-        if (!(ok = finalize(j + 1, false))) break;
-        fin_k = j + 2;
+        if (!(ok = issue_k(j + 1))) break;
+        nk = j + 2;
       }
-      if (j + kStages < T) {
-        // K stage of tile j is free once QK(j) is done
-        if (!(ok = wait_bounded(&bars->k_empty[j % kStages], (j / kStages) & 1, p.spin,
-                                abort_flag)))
-          break;
-        issue(j + kStages, false);
-        ++issued_k;
-      }
-      if (j + 1 < T) {
-        if (!(ok = finalize(j + 1, true))) break;
-        fin_v = j + 2;
-      }
-      if (j + kStages < T) {
-        // V stage of tile j is free once PV(j) is done
-        if (!(ok = wait_bounded(&bars->v_empty[j % kStages], (j / kStages) & 1, p.spin,
-                                abort_flag)))
-          break;
-        issue(j + kStages, true);
-        ++issued_v;
-      }
+      if (!(ok = issue_v(j))) break;
+      nv = j + 1;
     }
-    // never leave with TMA writes in flight
-    for (int j = fin_k; j < issued_k; ++j)
-      wait_bounded(&bars->k_full[j % kStages], (j / kStages) & 1, p.spin, abort_flag);
-    for (int j = fin_v; j < issued_v; ++j)
-      wait_bounded(&bars->v_full[j % kStages], (j / kStages) & 1, p.spin, abort_flag);
+    // never leave with TMA writes in flight: the last load of every stage has landed
+    for (int s = 0; s < kSK && s < nk; ++s) {
+      const int j = nk - 1 - ((nk - 1 - s) % kSK + kSK) % kSK;  // last tile issued to stage s
+      if (j >= 0) wait_bounded(&bars->k_full[s], (j / kSK) & 1, p.spin, abort_flag);
+    }
+    for (int s = 0; s < kSV && s < nv; ++s) {
+      const int j = nv - 1 - ((nv - 1 - s) % kSV + kSV) % kSV;
+      if (j >= 0) wait_bounded(&bars->v_full[s], (j / kSV) & 1, p.spin, abort_flag);
+    }
     wait_bounded(&bars->q_full, 0, p.spin, abort_flag);
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
@@ -308,7 +231,7 @@ attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const uint32_t idSt = idesc_bf16(kBM, 16, false);
       const uint32_t sQ = sbase + Lay::kQ;
       auto qk = [&](int j) {
-        const int s = j % kStages;
+        const int s = j % kSK;
         const uint32_t sK = sbase + Lay::kK + s * Lay::kTile;
         const uint32_t dS = tmem + ((j & 1) ? Lay::kS1 : Lay::kS0);
 #pragma unroll
@@ -320,24 +243,23 @@ attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         mma_commit(&bars->k_empty[s]);
       };
       bool ok = wait_bounded(&bars->q_full, 0, p.spin, abort_flag);
-      ok = ok && wait_bounded(&bars->k_ready[0], 0, p.spin, abort_flag);
+      ok = ok && wait_bounded(&bars->k_full[0], 0, p.spin, abort_flag);
       if (ok) {
         fence_after_sync();
         qk(0);
       }
       for (int j = 0; ok && j < T; ++j) {
         if (j + 1 < T) {
-          const int s1 = (j + 1) % kStages;
-          ok = wait_bounded(&bars->k_ready[s1], ((j + 1) / kStages) & 1, p.spin, abort_flag);
+          ok = wait_bounded(&bars->k_full[(j + 1) % kSK], ((j + 1) / kSK) & 1, p.spin, abort_flag);
           // S(j+1) overwrites the buffer that held P(j-1): PV(j-1) must be done
           if (ok && j >= 1) ok = wait_bounded(&bars->pv_done, (j - 1) & 1, p.spin, abort_flag);
           if (!ok) break;
           fence_after_sync();
           qk(j + 1);
         }
-        const int s = j % kStages;
+        const int s = j % kSV;
         ok = wait_bounded(&bars->p_full[j & 1], (j >> 1) & 1, p.spin, abort_flag) &&
-             wait_bounded(&bars->v_ready[s], (j / kStages) & 1, p.spin, abort_flag);
+             wait_bounded(&bars->v_full[s], (j / kSV) & 1, p.spin, abort_flag);
         if (!ok) break;
         fence_after_sync();
         const uint32_t tP = tmem + ((j & 1) ? Lay::kS1 : Lay::kS0);  // P(j), bf16 pairs
@@ -367,6 +289,8 @@ attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
     const bool seed_row =
         i < L && p.is_seed != nullptr && p.is_seed[(int64_t)b * L + i] != 0;
+    // rank among the sequence's masked rows (-1: not masked or no pass 2)
+    const int rank = (p.q_m != nullptr && i < L) ? p.mrank[(int64_t)b * L + i] : -1;
     const float c2 = p.scale_log2;
     float m = -INFINITY;
     bool ok = true;
@@ -512,8 +436,24 @@ attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           v.w = pack_bf16(o[c * 8 + 6] * inv, o[c * 8 + 7] * inv);
           dst[c] = v;
         }
-        p.lse[((int64_t)b * p.Hq + h) * L + i] = (m + log2f(l)) * kLn2;
+        const float lse2 = m + log2f(l);
+        p.lse[((int64_t)b * p.Hq + h) * L + i] = lse2 * kLn2;
         if (p.dout_part) p.dout_part[((int64_t)b * p.Hq + h) * L + i] = ln * inv;
+        if (rank >= 0) {
+          // pass 2's inputs for a still-masked row: its Q row (from the staged,
+          // swizzled tile; q_full completed long before) and its lse in log2 units
+          wait_bounded(&bars->q_full, 0, p.spin, abort_flag);
+          uint4* qd = reinterpret_cast<uint4*>(p.q_m + (((int64_t)b * L + rank) * p.Hq + h) * D);
+#pragma unroll
+          for (int c = 0; c < D / 8; ++c) {
+            uint4 v;
+            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                         : "r"(sbase + Lay::kQ + (c / 8) * kAtom + sw128(r, c & 7)));
+            qd[c] = v;
+          }
+          p.lse2_m[((int64_t)b * p.Hq + h) * p.Lp + rank] = lse2;
+        }
       }
     }
   }
@@ -527,30 +467,30 @@ attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
 // --------------------------------------------------------------------------- pass 2
 // d_in partials: one CTA per (128 key columns, kv head, sequence). The key tile
-// (drafting view: seed columns from the cache) stays in shared memory; the CTA
-// loops over the G query heads sharing this kv head and over tiles of 128
-// still-masked query rows (gathered). S^T = K Q_m^T puts one key column per
-// TMEM lane, so each consumer thread sums exp2(S * scale * log2e - lse2) over
-// its own column without any cross-thread reduction.
-//   warps 0-3  producers: warp 0 issues the key TMA and patches seed rows; all
-//              four gather masked query rows (plain loads, swizzled stores) and
-//              their lse (natural log -> log2 units) into a double buffer
-//   warp 4     MMA issuer
-//   warps 5-8  consumers (one key column each)
-constexpr int kP2Threads = 288;
+// of the drafting view stays in shared memory; the CTA loops over the G query
+// heads sharing this kv head and over tiles of 128 still-masked query rows,
+// which pass 1 left in rank order (q_m) together with their lse (lse2_m, log2
+// units). S^T = K Q_m^T puts one key column per TMEM lane, so each consumer
+// thread sums exp2(S * scale * log2e - lse2) over its own column without any
+// cross-thread reduction.
+//   warp 0     producer: TMA of the key tile, then per row tile a TMA of the
+//              Q_m tile and a bulk copy of its 128 lse values (double buffer)
+//   warp 1     MMA issuer
+//   warps 2-5  consumers (one key column each)
+constexpr int kP2Threads = 192;
 
 template <int D>
 struct P2Layout {
   static constexpr int kTile = (D / 64) * kAtom;
   static constexpr int kK = 0;
-  static constexpr int kQ = kK + kTile;               // two buffers
-  static constexpr int kLse = kQ + 2 * kTile;         // two buffers of 128 floats
+  static constexpr int kQ = kK + kTile;        // two buffers
+  static constexpr int kLse = kQ + 2 * kTile;  // two buffers of 128 floats
   static constexpr int kBar = kLse + 2 * 128 * 4;
-  static constexpr int kBytes = kBar + 256;
+  static constexpr int kBytes = kBar + 128;
 };
 
 struct P2Bars {
-  uint64_t k_full, k_ready;
+  uint64_t k_full;
   uint64_t q_full[2];
   uint64_t s_full[2];
   uint64_t c_done[2];
@@ -560,26 +500,25 @@ struct P2Bars {
 };
 
 struct P2Params {
-  const __nv_bfloat16 *q, *k_prev;
-  const uint32_t* seedbits;
-  const float* lse;
-  const int32_t *mrows, *mcount;
-  int L, Hq, Hkv;
+  const int32_t* mcount;
+  const float* lse2_m;  // [B, Hq, Lp]
+  int L, Hq, Hkv, Lp;
   float scale_log2;
   float* din_part;  // [B, Hkv, L]
   uint32_t spin;
 };
 
 template <int D>
-__global__ void __launch_bounds__(kP2Threads, 1)
-attn_p2_kernel(const __grid_constant__ CUtensorMap tmK, const P2Params p) {
+__global__ void __launch_bounds__(kP2Threads, 2)
+attn_p2_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQm,
+               const P2Params p) {
   using Lay = P2Layout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   P2Bars* bars = reinterpret_cast<P2Bars*>(smem + Lay::kBar);
   const uint32_t sbase = smem_u32(smem);
-  float* lse2 = reinterpret_cast<float*>(smem + Lay::kLse);
+  const float* lse2 = reinterpret_cast<const float*>(smem + Lay::kLse);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kt = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int L = p.L;
@@ -592,9 +531,8 @@ attn_p2_kernel(const __grid_constant__ CUtensorMap tmK, const P2Params p) {
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->k_full, 1);
-    mbar_init(&bars->k_ready, 1);
     for (int u = 0; u < 2; ++u) {
-      mbar_init(&bars->q_full[u], 128);
+      mbar_init(&bars->q_full[u], 1);
       mbar_init(&bars->s_full[u], 1);
       mbar_init(&bars->c_done[u], 4);
     }
@@ -602,7 +540,7 @@ attn_p2_kernel(const __grid_constant__ CUtensorMap tmK, const P2Params p) {
     bars->abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 4) {
+  if (warp == 1) {
     tmem_alloc(&bars->tmem_base, 256);
     tmem_relinquish();
   }
@@ -611,72 +549,47 @@ attn_p2_kernel(const __grid_constant__ CUtensorMap tmK, const P2Params p) {
   fence_after_sync();
   const uint32_t tmem = bars->tmem_base;
 
-  if (warp < 4) {
-    // ------------------------------------------------------------------ producers
-    const int pt = threadIdx.x;  // 0..127: the masked row this thread gathers
-    if (warp == 0) {
-      if (lane == 0) {
+  if (warp == 0) {
+    // ------------------------------------------------------------------ producer
+    if (lane == 0) {
+      if (NT > 0) {
         mbar_expect_tx(&bars->k_full, Lay::kTile);
 #pragma unroll
         for (int ac = 0; ac < D / 64; ++ac)
           tma_load_4d(smem + Lay::kK + ac * kAtom, &tmK, ac * 64, g, col0, b, &bars->k_full);
       }
-      const int W = (L + 31) / 32;
-      uint32_t seedword = 0;
-      if (lane < 4 && kt * 4 + lane < W) seedword = p.seedbits[(int64_t)b * W + kt * 4 + lane];
-      if (wait_bounded(&bars->k_full, 0, p.spin, abort_flag)) {
+      int issued = 0;
+      for (int t = 0; t < NT; ++t) {
+        const int u = t & 1;
+        // buffer u is free once the consumers are done with tile t-2 (its QK is done too)
+        if (t >= 2 && !wait_bounded(&bars->c_done[u], ((t >> 1) - 1) & 1, p.spin, abort_flag)) break;
+        const int hh = g * G + t / nrt;
+        const int m0 = (t % nrt) * 128;
+        mbar_expect_tx(&bars->q_full[u], Lay::kTile + 128 * 4);
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          uint32_t bits = __shfl_sync(0xffffffffu, seedword, w);
-          while (bits) {
-            const int r = w * 32 + __ffs(bits) - 1;
-            bits &= bits - 1;
-            if (lane < D / 8) {
-              const uint4 val =
-                  ldg16(p.k_prev + (((int64_t)b * L + col0 + r) * p.Hkv + g) * D + lane * 8);
-              st_shared_v4(sbase + Lay::kK + (lane / 8) * kAtom + sw128(r, lane & 7), val.x,
-                           val.y, val.z, val.w);
-            }
-          }
-        }
-        fence_proxy_async();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->k_ready);
+        for (int ac = 0; ac < D / 64; ++ac)
+          tma_load_4d(smem + Lay::kQ + u * Lay::kTile + ac * kAtom, &tmQm, ac * 64, hh, m0, b,
+                      &bars->q_full[u]);
+        bulk_load(smem + Lay::kLse + u * 512, p.lse2_m + ((int64_t)b * p.Hq + hh) * p.Lp + m0, 512,
+                  &bars->q_full[u]);
+        issued = t + 1;
       }
+      // never leave with copies in flight
+      if (NT > 0) wait_bounded(&bars->k_full, 0, p.spin, abort_flag);
+      for (int t = issued - 2 < 0 ? 0 : issued - 2; t < issued; ++t)
+        wait_bounded(&bars->q_full[t & 1], (t >> 1) & 1, p.spin, abort_flag);
     }
-    for (int t = 0; t < NT; ++t) {
-      const int u = t & 1;
-      if (t >= 2 && !wait_bounded(&bars->c_done[u], ((t >> 1) - 1) & 1, p.spin, abort_flag)) break;
-      const int hh = g * G + t / nrt;
-      const int m = (t % nrt) * 128 + pt;
-      const uint32_t qb = sbase + Lay::kQ + u * Lay::kTile;
-      if (m < M) {
-        const int pos = p.mrows[(int64_t)b * L + m];
-        const __nv_bfloat16* src = p.q + (((int64_t)b * L + pos) * p.Hq + hh) * D;
-#pragma unroll
-        for (int c = 0; c < D / 8; ++c) {
-          const uint4 val = ldg16(src + c * 8);
-          st_shared_v4(qb + (c / 8) * kAtom + sw128(pt, c & 7), val.x, val.y, val.z, val.w);
-        }
-        lse2[u * 128 + pt] = p.lse[((int64_t)b * p.Hq + hh) * L + pos] * kLog2e;
-      } else {
-#pragma unroll
-        for (int c = 0; c < D / 8; ++c)
-          st_shared_v4(qb + (c / 8) * kAtom + sw128(pt, c & 7), 0u, 0u, 0u, 0u);
-        lse2[u * 128 + pt] = INFINITY;
-      }
-      fence_proxy_async();
-      mbar_arrive(&bars->q_full[u]);
-    }
-  } else if (warp == 4) {
+    __syncwarp();
+  } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idS = idesc_bf16(kBM, kBN, false);
       const uint32_t sK = sbase + Lay::kK;
-      bool ok = NT == 0 || wait_bounded(&bars->k_ready, 0, p.spin, abort_flag);
+      bool ok = NT == 0 || wait_bounded(&bars->k_full, 0, p.spin, abort_flag);
       for (int t = 0; ok && t < NT; ++t) {
         const int u = t & 1;
         ok = wait_bounded(&bars->q_full[u], (t >> 1) & 1, p.spin, abort_flag);
+        // S buffer u held tile t-2: its consumers must be done with it
         if (ok && t >= 2) ok = wait_bounded(&bars->c_done[u], ((t >> 1) - 1) & 1, p.spin, abort_flag);
         if (!ok) break;
         fence_after_sync();
@@ -703,7 +616,9 @@ attn_p2_kernel(const __grid_constant__ CUtensorMap tmK, const P2Params p) {
     bool ok = true;
     for (int t = 0; t < NT; ++t) {
       const int u = t & 1;
-      ok = wait_bounded(&bars->s_full[u], (t >> 1) & 1, p.spin, abort_flag);
+      // lse values land with the Q tile; S(t) done implies q_full(t) completed
+      ok = wait_bounded(&bars->s_full[u], (t >> 1) & 1, p.spin, abort_flag) &&
+           wait_bounded(&bars->q_full[u], (t >> 1) & 1, p.spin, abort_flag);
       if (!ok) break;
       fence_after_sync();
       float s[kBN];
@@ -716,14 +631,30 @@ attn_p2_kernel(const __grid_constant__ CUtensorMap tmK, const P2Params p) {
       }
       tmem_wait_ld();
       const float4* lv = reinterpret_cast<const float4*>(lse2 + u * 128);
+      const int nvalid = min(128, M - (t % nrt) * 128);  // rows past the count are unset
       float a0 = 0.f, a1 = 0.f;
+      if (nvalid == 128) {
 #pragma unroll
-      for (int c4 = 0; c4 < kBN / 4; ++c4) {
-        const float4 l4 = lv[c4];
-        a0 += fast_exp2(fmaf(s[4 * c4 + 0], c2, -l4.x));
-        a1 += fast_exp2(fmaf(s[4 * c4 + 1], c2, -l4.y));
-        a0 += fast_exp2(fmaf(s[4 * c4 + 2], c2, -l4.z));
-        a1 += fast_exp2(fmaf(s[4 * c4 + 3], c2, -l4.w));
+        for (int c4 = 0; c4 < kBN / 4; ++c4) {
+          const float4 l4 = lv[c4];
+          a0 += fast_exp2(fmaf(s[4 * c4 + 0], c2, -l4.x));
+          a1 += fast_exp2(fmaf(s[4 * c4 + 1], c2, -l4.y));
+          a0 += fast_exp2(fmaf(s[4 * c4 + 2], c2, -l4.z));
+          a1 += fast_exp2(fmaf(s[4 * c4 + 3], c2, -l4.w));
+        }
+      } else {
+#pragma unroll
+        for (int c4 = 0; c4 < kBN / 4; ++c4) {
+          const float4 l4 = lv[c4];
+          const float l[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = 4 * c4 + e;
+            const float x = c < nvalid ? fmaf(s[c], c2, -l[e]) : -INFINITY;
+            if (e & 1) a1 += fast_exp2(x);
+            else a0 += fast_exp2(x);
+          }
+        }
       }
       acc += a0 + a1;
       fence_before_sync();
@@ -734,7 +665,7 @@ attn_p2_kernel(const __grid_constant__ CUtensorMap tmK, const P2Params p) {
   }
   fence_before_sync();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == 1) {
     fence_after_sync();
     tmem_dealloc(tmem, 256);
   }
@@ -768,28 +699,14 @@ bool make_map(CUtensorMap* map, const void* base, int D, int H, int L, int B) {
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Rows of the step t-1 cache: box = one whole head row (D elements), no swizzle.
-bool make_row_map(CUtensorMap* map, const void* base, int D, int H, int L, int B) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)L, (cuuint64_t)B};
-  cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)L * H * D * 2};
-  cuuint32_t box[4] = {(cuuint32_t)D, 1, 1, 1};
-  cuuint32_t estr[4] = {1, 1, 1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int D>
-cudaError_t launch_p1(const AttnArgs& a, cudaStream_t stream) {
-  CUtensorMap tq, tk, tv, tkp, tvp;
-  // without seeds the cache maps are never read; point them at the current K/V
-  const void* kp = a.is_seed ? a.k_prev : a.k_cur;
-  const void* vp = a.is_seed ? a.v_prev : a.v_cur;
-  if (!make_map(&tq, a.q, D, a.Hq, a.L, a.B) || !make_map(&tk, a.k_cur, D, a.Hkv, a.L, a.B) ||
-      !make_map(&tv, a.v_cur, D, a.Hkv, a.L, a.B) ||
-      !make_row_map(&tkp, kp, D, a.Hkv, a.L, a.B) || !make_row_map(&tvp, vp, D, a.Hkv, a.L, a.B))
+cudaError_t launch_p1(const AttnArgs& a, bool pass2, cudaStream_t stream) {
+  CUtensorMap tq, tk, tv;
+  // without seeds the drafting view is the current input itself
+  const void* kv = a.is_seed ? a.k_view : a.k_cur;
+  const void* vv = a.is_seed ? a.v_view : a.v_cur;
+  if (!make_map(&tq, a.q, D, a.Hq, a.L, a.B) || !make_map(&tk, kv, D, a.Hkv, a.L, a.B) ||
+      !make_map(&tv, vv, D, a.Hkv, a.L, a.B))
     return cudaErrorInvalidValue;
   const int smem = P1Layout<D>::kBytes + 1024;
   static int configured[64] = {};
@@ -804,29 +721,32 @@ cudaError_t launch_p1(const AttnArgs& a, cudaStream_t stream) {
   p.q = static_cast<const __nv_bfloat16*>(a.q);
   p.k_cur = static_cast<const __nv_bfloat16*>(a.k_cur);
   p.v_cur = static_cast<const __nv_bfloat16*>(a.v_cur);
-  p.k_prev = static_cast<const __nv_bfloat16*>(a.k_prev);
-  p.v_prev = static_cast<const __nv_bfloat16*>(a.v_prev);
   p.is_seed = a.is_seed;
   p.is_new = a.is_new;
-  p.seedbits = a.seedbits;
   p.newbits = a.newbits;
+  p.mrank = a.mrank;
   p.L = a.L;
   p.Hq = a.Hq;
   p.Hkv = a.Hkv;
+  p.Lp = a.Lp;
   p.scale_log2 = a.scale * kLog2e;
   p.out = static_cast<__nv_bfloat16*>(a.out);
   p.lse = a.lse;
   p.dout_part = a.dout_part;
+  p.q_m = pass2 ? static_cast<__nv_bfloat16*>(a.q_m) : nullptr;
+  p.lse2_m = a.lse2_m;
   p.spin = spin_limit();
   dim3 grid((a.L + kBM - 1) / kBM, a.Hq, a.B);
-  attn_p1_kernel<D><<<grid, kP1Threads, smem, stream>>>(tq, tk, tv, tkp, tvp, p);
+  attn_p1_kernel<D><<<grid, kP1Threads, smem, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
 
 template <int D>
 cudaError_t launch_p2(const AttnArgs& a, cudaStream_t stream) {
-  CUtensorMap tk;
-  if (!make_map(&tk, a.k_cur, D, a.Hkv, a.L, a.B)) return cudaErrorInvalidValue;
+  CUtensorMap tk, tqm;
+  const void* kv = a.is_seed ? a.k_view : a.k_cur;
+  if (!make_map(&tk, kv, D, a.Hkv, a.L, a.B) || !make_map(&tqm, a.q_m, D, a.Hq, a.L, a.B))
+    return cudaErrorInvalidValue;
   const int smem = P2Layout<D>::kBytes + 1024;
   static int configured[64] = {};
   const int dev = device_info().device;
@@ -837,20 +757,17 @@ cudaError_t launch_p2(const AttnArgs& a, cudaStream_t stream) {
     configured[dev & 63] = 1;
   }
   P2Params p;
-  p.q = static_cast<const __nv_bfloat16*>(a.q);
-  p.k_prev = static_cast<const __nv_bfloat16*>(a.k_prev);
-  p.seedbits = a.seedbits;
-  p.lse = a.lse;
-  p.mrows = a.mrows;
   p.mcount = a.mcount;
+  p.lse2_m = a.lse2_m;
   p.L = a.L;
   p.Hq = a.Hq;
   p.Hkv = a.Hkv;
+  p.Lp = a.Lp;
   p.scale_log2 = a.scale * kLog2e;
   p.din_part = a.din_part;
   p.spin = spin_limit();
   dim3 grid((a.L + kBN - 1) / kBN, a.Hkv, a.B);
-  attn_p2_kernel<D><<<grid, kP2Threads, smem, stream>>>(tk, p);
+  attn_p2_kernel<D><<<grid, kP2Threads, smem, stream>>>(tk, tqm, p);
   return cudaGetLastError();
 }
 
@@ -860,9 +777,10 @@ cudaError_t launch_p2(const AttnArgs& a, cudaStream_t stream) {
 cudaError_t launch_attention_tc(const AttnArgs& a, cudaStream_t stream, bool* handled,
                                 int* din_slices) {
   *handled = true;
-  cudaError_t err = a.d == 64 ? launch_p1<64>(a, stream) : launch_p1<128>(a, stream);
+  const bool pass2 = a.d_in != nullptr && a.is_masked != nullptr;
+  cudaError_t err = a.d == 64 ? launch_p1<64>(a, pass2, stream) : launch_p1<128>(a, pass2, stream);
   if (err != cudaSuccess) return err;
-  if (a.d_in && a.is_masked) {
+  if (pass2) {
     err = a.d == 64 ? launch_p2<64>(a, stream) : launch_p2<128>(a, stream);
     *din_slices = a.Hkv;
   }

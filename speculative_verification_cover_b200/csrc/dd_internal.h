@@ -38,13 +38,21 @@ struct AttnArgs {
   int32_t* mcount;      // [B]
   uint32_t* seedbits;   // [B, ceil(L/32)] packed is_seed
   uint32_t* newbits;    // [B, ceil(L/32)] packed is_new
+  int32_t* mrank;       // [B, L] rank of a masked row among its sequence's masked rows, else -1
+  // tensor-core path only (bf16)
+  void *k_view, *v_view;  // [B, L, Hkv, d] drafting view: seed rows from the cache, others current
+  void* q_m;              // [B, L, Hq, d] masked query rows in rank order (rows >= count unset)
+  float* lse2_m;          // [B, Hq, Lp] lse (log2 units) of masked rows in rank order
+  int Lp;                 // L rounded up to 128
 };
 
 // Workspace layout shared by the entry point and the kernels.
 struct AttnWorkspace {
-  size_t dout_off, din_off, mrows_off, mcount_off, seedbits_off, newbits_off, total;
+  size_t dout_off, din_off, mrows_off, mcount_off, seedbits_off, newbits_off, mrank_off;
+  size_t kview_off, vview_off, qm_off, lse2m_off, total;
+  int Lp;
 };
-AttnWorkspace attn_workspace_layout(int B, int L, int Hq);
+AttnWorkspace attn_workspace_layout(int B, int L, int Hq, int Hkv, int d);
 
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t stream);
 
