@@ -295,7 +295,9 @@ attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     float m = -INFINITY;
     bool ok = true;
     for (int j = 0; j < T; ++j) {
-      ok = wait_bounded(&bars->s_full[j & 1], (j >> 1) & 1, p.spin, abort_flag);
+      // warp-uniform outcome: the tcgen05 loads below are warp-wide
+      ok = __all_sync(0xffffffffu,
+                      wait_bounded(&bars->s_full[j & 1], (j >> 1) & 1, p.spin, abort_flag));
       if (!ok) break;
       fence_after_sync();
       float s[kBN];
@@ -336,7 +338,8 @@ attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const bool resc = need && j > 0 && m != -INFINITY;
       if (__any_sync(0xffffffffu, resc)) {
         // O (and the statistics columns) may only be rescaled once PV(j-1) is done
-        ok = wait_bounded(&bars->pv_done, (j - 1) & 1, p.spin, abort_flag);
+        ok = __all_sync(0xffffffffu,
+                        wait_bounded(&bars->pv_done, (j - 1) & 1, p.spin, abort_flag));
         if (!ok) break;
         fence_after_sync();
         const float f = resc ? exp2f(m - m_new) : 1.f;
@@ -375,7 +378,7 @@ attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     }
     // Warps may be a tile apart, so pv_done's parity cannot tell PV(T-1) from
     // PV(T-3) here; drain completes once, after every tensor-core operation.
-    if (ok) ok = wait_bounded(&bars->drain, 0, p.spin, abort_flag);
+    if (ok) ok = __all_sync(0xffffffffu, wait_bounded(&bars->drain, 0, p.spin, abort_flag));
     if (ok) {
       fence_after_sync();
       float o[D];
@@ -617,8 +620,9 @@ attn_p2_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
     for (int t = 0; t < NT; ++t) {
       const int u = t & 1;
       // lse values land with the Q tile; S(t) done implies q_full(t) completed
-      ok = wait_bounded(&bars->s_full[u], (t >> 1) & 1, p.spin, abort_flag) &&
-           wait_bounded(&bars->q_full[u], (t >> 1) & 1, p.spin, abort_flag);
+      ok = __all_sync(0xffffffffu,
+                      wait_bounded(&bars->s_full[u], (t >> 1) & 1, p.spin, abort_flag) &&
+                          wait_bounded(&bars->q_full[u], (t >> 1) & 1, p.spin, abort_flag));
       if (!ok) break;
       fence_after_sync();
       float s[kBN];
@@ -708,15 +712,6 @@ cudaError_t launch_p1(const AttnArgs& a, bool pass2, cudaStream_t stream) {
   if (!make_map(&tq, a.q, D, a.Hq, a.L, a.B) || !make_map(&tk, kv, D, a.Hkv, a.L, a.B) ||
       !make_map(&tv, vv, D, a.Hkv, a.L, a.B))
     return cudaErrorInvalidValue;
-  const int smem = P1Layout<D>::kBytes + 1024;
-  static int configured[64] = {};
-  const int dev = device_info().device;
-  if (!configured[dev & 63]) {
-    cudaError_t e = cudaFuncSetAttribute(attn_p1_kernel<D>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    configured[dev & 63] = 1;
-  }
   P1Params p;
   p.q = static_cast<const __nv_bfloat16*>(a.q);
   p.k_cur = static_cast<const __nv_bfloat16*>(a.k_cur);
@@ -736,6 +731,15 @@ cudaError_t launch_p1(const AttnArgs& a, bool pass2, cudaStream_t stream) {
   p.q_m = pass2 ? static_cast<__nv_bfloat16*>(a.q_m) : nullptr;
   p.lse2_m = a.lse2_m;
   p.spin = spin_limit();
+  const DeviceInfo& di = device_info();
+  const int smem = P1Layout<D>::kBytes + 1024;
+  static int configured[64] = {};
+  if (!configured[di.device & 63]) {
+    cudaError_t e = cudaFuncSetAttribute(attn_p1_kernel<D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    configured[di.device & 63] = 1;
+  }
   dim3 grid((a.L + kBM - 1) / kBM, a.Hq, a.B);
   attn_p1_kernel<D><<<grid, kP1Threads, smem, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();

@@ -23,7 +23,17 @@ __device__ __forceinline__ void record_error(unsigned int code) {
 
 // ---------------------------------------------------------------------------
 // mbarrier helpers (shared::cta). Every wait is bounded by `limit`
-// iterations; on expiry it records DD_ERR_TIMEOUT and returns false.
+// iterations and by kWaitNs of wall time (a try_wait may suspend the thread
+// for a while, so iterations alone do not bound the time); on expiry it
+// records DD_ERR_TIMEOUT and returns false.
+constexpr uint64_t kWaitNs = 2000000000ull;
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -32,21 +42,29 @@ __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
 }
 
+// A waiting thread is suspended by the hardware until the phase completes or
+// the hint (ns) runs out, so waiting warps take no issue slots from the warps
+// that share their SM sub-partition.
+constexpr uint32_t kSuspendHintNs = 1000000u;
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t phase) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(phase)
+      : "r"(smem_u32(bar)), "r"(phase), "r"(kSuspendHintNs)
       : "memory");
   return ok != 0;
 }
 
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t phase, uint32_t limit) {
-  for (uint32_t it = 0; it < limit; ++it) {
+  if (mbar_try_wait(bar, phase)) return true;
+  const uint64_t t0 = global_ns();
+  for (uint32_t it = 1; it < limit; ++it) {
     if (mbar_try_wait(bar, phase)) return true;
+    if (global_ns() - t0 > kWaitNs) break;
   }
   record_error(DD_ERR_TIMEOUT);
   return false;

@@ -216,9 +216,12 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 // Bounded wait executed by every lane of a warp (each lane polls).
 __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t phase, uint32_t limit,
                                              volatile int* abort_flag) {
-  for (uint32_t it = 0; it < limit; ++it) {
+  if (mbar_try_wait(bar, phase)) return true;
+  const uint64_t t0 = global_ns();
+  for (uint32_t it = 1; it < limit; ++it) {
     if (mbar_try_wait(bar, phase)) return true;
-    if ((it & 1023u) == 1023u && *abort_flag) return false;
+    if (*abort_flag) return false;
+    if (global_ns() - t0 > kWaitNs) break;
   }
   record_error(DD_ERR_TIMEOUT);
   *abort_flag = 1;

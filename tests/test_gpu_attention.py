@@ -72,6 +72,10 @@ CASES = [
     (3, 257, 8, 8, 128, torch.bfloat16),
     (1, 1, 1, 1, 128, torch.bfloat16),
     (1, 2, 2, 1, 64, torch.float32),
+    # many heads per kv head with a ragged L (rows past L in the last query
+    # tile of every head), and d = 64 with 16-way grouping
+    (2, 333, 80, 8, 128, torch.bfloat16),
+    (1, 600, 128, 16, 64, torch.bfloat16),
 ]
 
 
