@@ -7,13 +7,13 @@
 // Pass 1, one CTA per (128 query rows, head, sequence), warp-specialised:
 //   warp 0      producer: TMA loads of the Q tile and of K / V tiles of the
 //               view (128 columns; K and V have their own stage rings), and the
-//               tile's "newly written" flags as row 1 of a small B operand whose
-//               rows are [1, is_new, 0, ...].
+//               tile's "newly written" flags into a 16-column block next to the
+//               V tile whose key rows read [1, is_new(key), 0, ...].
 //   warp 1      MMA issuer (one thread): S = Q K^T into a double-buffered TMEM
-//               accumulator; O += P V and [l, l_new] += P [1, is_new]^T with P
-//               read from TMEM, i.e. the row sum and the mass on newly written
-//               columns come out of the tensor core with the same bf16 P that
-//               weights V.
+//               accumulator; [O | l | l_new] += P [V | 1 | is_new] as one MMA of
+//               N = D + 16 with P read from TMEM, i.e. the row sum and the mass on
+//               newly written columns come out of the tensor core with the same
+//               bf16 P that weights V, at the cost of 16 extra output columns.
 //   warps 2-5   softmax (one thread per query row = TMEM lane): online max with
 //               a lazy rescale (O is rescaled in TMEM only when the running max
 //               grows by more than 2^8), P = exp2(S*scale*log2e - m) as bf16
@@ -36,7 +36,7 @@ using namespace tc;
 
 constexpr int kBM = 128;
 constexpr int kBN = 128;
-constexpr int kSK = 3;  // K stages
+constexpr int kSK = 2;  // K stages
 constexpr int kSV = 2;  // V stages
 constexpr int kP1Threads = 192;
 constexpr uint32_t kTmemCols = 512;
@@ -47,11 +47,13 @@ struct P1Layout {
   static constexpr int kTile = (D / 64) * kAtom;  // 128 x D bf16
   static constexpr int kQ = 0;
   static constexpr int kK = kQ + kTile;
+  // A V stage is the V tile plus one more 64-column swizzle atom whose first
+  // 16 columns are [1, is_new(key), 0...]: PV with N = D + 16 then yields O and
+  // the statistics [l, l_new] together.
+  static constexpr int kVStage = kTile + kAtom;
   static constexpr int kV = kK + kSK * kTile;
-  static constexpr int kB2 = kV + kSV * kTile;
-  static constexpr int kB2Bytes = 2 * 16 * 128;  // 16 rows x 128 columns bf16
   // packed newly-written flags of the whole sequence
-  static constexpr int kNew = kB2 + kSV * kB2Bytes;
+  static constexpr int kNew = kV + kSV * kVStage;
   static constexpr int kNewWords = kTcMaxL / 32;
   static constexpr int kBar = kNew + kNewWords * 4;
   static constexpr int kBytes = kBar + 256;
@@ -131,15 +133,12 @@ attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     tmem_alloc(&bars->tmem_base, kTmemCols);
     tmem_relinquish();
   }
-  // constant rows of the [1, is_new, 0...] operand: row 0 = ones, rows 2..15 = 0
+  // the statistics atoms start at zero (chunk 0 of each row is rewritten per tile)
   if (warp >= 2) {
     const int t = threadIdx.x - 64;  // 0..127
-    for (int idx = t; idx < kSV * 2 * 16 * 8; idx += 128) {
-      const int s = idx / (2 * 16 * 8), rem = idx % (2 * 16 * 8);
-      const int ac = rem / (16 * 8), row = (rem / 8) % 16, c = rem % 8;
-      const uint32_t one = 0x3F803F80u;  // two bf16 1.0
-      const uint32_t v = row == 0 ? one : 0u;
-      st_shared_v4(sbase + Lay::kB2 + s * Lay::kB2Bytes + ac * 2048 + sw128(row, c), v, v, v, v);
+    for (int idx = t; idx < kSV * 128 * 8; idx += 128) {
+      const int s = idx / (128 * 8), row = (idx / 8) % 128, c = idx % 8;
+      st_shared_v4(sbase + Lay::kV + s * Lay::kVStage + Lay::kTile + sw128(row, c), 0u, 0u, 0u, 0u);
     }
     fence_proxy_async();
   }
@@ -178,17 +177,15 @@ attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const int s = j % kSV;
       if (j >= kSV && !wait_bounded(&bars->v_empty[s], ((j / kSV) - 1) & 1, p.spin, abort_flag))
         return false;
-      if (lane < 16) {
-        // row 1 of the statistics operand: the tile's newly-written flags
-        const int wi = j * 4 + lane / 4;
-        const uint32_t byte = ((wi < W ? neww[wi] : 0u) >> ((lane & 3) * 8)) & 0xFFu;
-        uint32_t w4[4];
+      {
+        // statistics columns of key row r: [1, is_new(r), 0, ...] (rows = keys)
+        const uint32_t atom = sbase + Lay::kV + s * Lay::kVStage + Lay::kTile;
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-          w4[e] = ((byte >> (2 * e)) & 1u ? 0x3F80u : 0u) |
-                  ((byte >> (2 * e + 1)) & 1u ? 0x3F800000u : 0u);
-        st_shared_v4(sbase + Lay::kB2 + s * Lay::kB2Bytes + (lane / 8) * 2048 + sw128(1, lane & 7),
-                     w4[0], w4[1], w4[2], w4[3]);
+        for (int rr = 0; rr < 4; ++rr) {
+          const int wi = j * 4 + rr;
+          const bool nw = wi < W && ((neww[wi] >> lane) & 1u);
+          st_shared_v4(atom + sw128(rr * 32 + lane, 0), nw ? 0x3F803F80u : 0x00003F80u, 0u, 0u, 0u);
+        }
       }
       fence_proxy_async();
       __syncwarp();
@@ -196,7 +193,7 @@ attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         mbar_expect_tx(&bars->v_full[s], Lay::kTile);
 #pragma unroll
         for (int ac = 0; ac < D / 64; ++ac)
-          tma_load_4d(smem + Lay::kV + s * Lay::kTile + ac * kAtom, &tmV, ac * 64, g, j * kBN, b,
+          tma_load_4d(smem + Lay::kV + s * Lay::kVStage + ac * kAtom, &tmV, ac * 64, g, j * kBN, b,
                       &bars->v_full[s]);
       }
       return true;
@@ -227,8 +224,7 @@ attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idS = idesc_bf16(kBM, kBN, false);
-      const uint32_t idO = idesc_bf16(kBM, D, true);
-      const uint32_t idSt = idesc_bf16(kBM, 16, false);
+      const uint32_t idO = idesc_bf16(kBM, D + 16, true);  // O and [l, l_new]
       const uint32_t sQ = sbase + Lay::kQ;
       auto qk = [&](int j) {
         const int s = j % kSK;
@@ -263,16 +259,11 @@ attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (!ok) break;
         fence_after_sync();
         const uint32_t tP = tmem + ((j & 1) ? Lay::kS1 : Lay::kS0);  // P(j), bf16 pairs
-        const uint32_t sV = sbase + Lay::kV + s * Lay::kTile;
-        const uint32_t sB2 = sbase + Lay::kB2 + s * Lay::kB2Bytes;
+        const uint32_t sV = sbase + Lay::kV + s * Lay::kVStage;
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
+        for (int kk = 0; kk < kBN / 16; ++kk)
           mma_bf16_ts(tmem + Lay::kO, tP + kk * 8, desc_mnmajor_sw128(sV + kk * 16 * 128, kAtom),
-                      idO, acc);
-          mma_bf16_ts(tmem + Lay::kSt, tP + kk * 8,
-                      desc_kmajor_sw128(sB2 + (kk / 4) * 2048 + (kk % 4) * 32), idSt, acc);
-        }
+                      idO, (j > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&bars->pv_done);
         mma_commit(&bars->v_empty[s]);
       }
