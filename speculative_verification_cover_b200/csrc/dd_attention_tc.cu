@@ -313,16 +313,18 @@ attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         for (int c = 0; c < kBN; ++c)
           if (c == r) s[c] = -INFINITY;
       }
-      // row maximum: eight independent chains, then a tree (short dependency chain)
+      // row maximum: eight independent chains of three-input maxima, then a tree
       float pm[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) pm[e] = s[e];
+      for (int e = 0; e < 8; ++e) pm[e] = fmax3(s[e], s[8 + e], s[16 + e]);
+      static_assert((kBN - 24) % 16 == 8, "chain schedule assumes 128 columns");
 #pragma unroll
-      for (int c = 8; c < kBN; c += 8)
+      for (int c = 24; c + 16 <= kBN; c += 16)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) pm[e] = fmaxf(pm[e], s[c + e]);
-      float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
-                       fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+        for (int e = 0; e < 8; ++e) pm[e] = fmax3(pm[e], s[c + e], s[c + 8 + e]);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) pm[e] = fmaxf(pm[e], s[kBN - 8 + e]);
+      float mx = fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
       mx *= c2;
       const bool need = mx > m + 8.f;
       const float m_new = need ? mx : m;
@@ -346,9 +348,11 @@ attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         tmem_wait_st();
       }
       m = m_new;
-      const bool live = m != -INFINITY;
       // P = exp2(S * scale * log2e - m) as bf16 pairs over the first 64 columns of
       // this tile's S buffer (already read into registers): the A operand of PV.
+      // While every score so far is masked (m = -inf) all of S is -inf and a zero
+      // reference gives exp2(-inf) = 0 without a per-element select.
+      const float mref = m == -INFINITY ? 0.f : m;
       const uint32_t scol = (j & 1) ? Lay::kS1 : Lay::kS0;
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
@@ -356,8 +360,8 @@ attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
           const int c = half * 64 + 2 * e;
-          const float a = live ? fast_exp2(fmaf(s[c], c2, -m)) : 0.f;
-          const float bb = live ? fast_exp2(fmaf(s[c + 1], c2, -m)) : 0.f;
+          const float a = fast_exp2(fmaf(s[c], c2, -mref));
+          const float bb = fast_exp2(fmaf(s[c + 1], c2, -mref));
           w[e] = pack_bf16(a, bb);
         }
         tmem_st32u(tl + scol + half * 32, w);
@@ -616,38 +620,45 @@ attn_p2_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
                           wait_bounded(&bars->q_full[u], (t >> 1) & 1, p.spin, abort_flag));
       if (!ok) break;
       fence_after_sync();
-      float s[kBN];
-#pragma unroll
-      for (int q = 0; q < kBN / 32; ++q) {
-        float tt[32];
-        tmem_ld32(tl + u * 128 + q * 32, tt);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) s[q * 32 + e] = tt[e];
-      }
-      tmem_wait_ld();
-      const float4* lv = reinterpret_cast<const float4*>(lse2 + u * 128);
       const int nvalid = min(128, M - (t % nrt) * 128);  // rows past the count are unset
       float a0 = 0.f, a1 = 0.f;
-      if (nvalid == 128) {
+      // two halves of 64 query rows (TMEM columns) each, to keep registers down
 #pragma unroll
-        for (int c4 = 0; c4 < kBN / 4; ++c4) {
-          const float4 l4 = lv[c4];
-          a0 += fast_exp2(fmaf(s[4 * c4 + 0], c2, -l4.x));
-          a1 += fast_exp2(fmaf(s[4 * c4 + 1], c2, -l4.y));
-          a0 += fast_exp2(fmaf(s[4 * c4 + 2], c2, -l4.z));
-          a1 += fast_exp2(fmaf(s[4 * c4 + 3], c2, -l4.w));
+      for (int hq = 0; hq < 2; ++hq) {
+        float s[64];
+        {
+          float t0[32], t1[32];
+          tmem_ld32(tl + u * 128 + hq * 64, t0);
+          tmem_ld32(tl + u * 128 + hq * 64 + 32, t1);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            s[e] = t0[e];
+            s[32 + e] = t1[e];
+          }
         }
-      } else {
+        const float4* lv = reinterpret_cast<const float4*>(lse2 + u * 128 + hq * 64);
+        if (nvalid == 128) {
 #pragma unroll
-        for (int c4 = 0; c4 < kBN / 4; ++c4) {
-          const float4 l4 = lv[c4];
-          const float l[4] = {l4.x, l4.y, l4.z, l4.w};
+          for (int c4 = 0; c4 < 16; ++c4) {
+            const float4 l4 = lv[c4];
+            a0 += fast_exp2(fmaf(s[4 * c4 + 0], c2, -l4.x));
+            a1 += fast_exp2(fmaf(s[4 * c4 + 1], c2, -l4.y));
+            a0 += fast_exp2(fmaf(s[4 * c4 + 2], c2, -l4.z));
+            a1 += fast_exp2(fmaf(s[4 * c4 + 3], c2, -l4.w));
+          }
+        } else {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int c = 4 * c4 + e;
-            const float x = c < nvalid ? fmaf(s[c], c2, -l[e]) : -INFINITY;
-            if (e & 1) a1 += fast_exp2(x);
-            else a0 += fast_exp2(x);
+          for (int c4 = 0; c4 < 16; ++c4) {
+            const float4 l4 = lv[c4];
+            const float l[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int c = hq * 64 + 4 * c4 + e;
+              const float x = c < nvalid ? fmaf(s[4 * c4 + e], c2, -l[e]) : -INFINITY;
+              if (e & 1) a1 += fast_exp2(x);
+              else a0 += fast_exp2(x);
+            }
           }
         }
       }
