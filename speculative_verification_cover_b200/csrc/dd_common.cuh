@@ -107,6 +107,27 @@ __device__ __forceinline__ float gumbel_from_word(uint32_t w) {
   return -__logf(e);
 }
 
+// An upper bound of gumbel_from_word(w) as computed above (its fp32 result),
+// cheap enough to screen every entry: -ln(-ln U) <= -ln(1 - U) since
+// -ln U >= 1 - U on (0, 1). With k = w >> 9, 1 - U = (j + 1/2) 2^-23 exactly for
+// j = 2^23 - 1 - k, so -ln(1 - U) = ln2 (23 - log2(j + 1/2)); j + 1/2 is formed
+// exactly from the float with bits (2^23 + j) minus (2^23 - 1/2). The 0.01
+// margin covers the approximate log2 here (about 4e-6 absolute) and the fp32
+// rounding of the exact path (about 1e-5): the bound is never below it.
+__device__ __forceinline__ float gumbel_bound_from_word(uint32_t w) {
+  const float jh = __uint_as_float((w >> 9) ^ 0x4B7FFFFFu) - 8388607.5f;
+  return fmaf(__log2f(jh), -0.69314718f, 23.f * 0.69314718f + 0.01f);
+}
+
+// Monotone map of floats (no NaN) onto signed integers, for integer max reductions.
+__device__ __forceinline__ int float_to_ordered(float x) {
+  const int i = __float_as_int(x);
+  return i >= 0 ? i : i ^ 0x7FFFFFFF;
+}
+__device__ __forceinline__ float ordered_to_float(int i) {
+  return __int_as_float(i >= 0 ? i : i ^ 0x7FFFFFFF);
+}
+
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }

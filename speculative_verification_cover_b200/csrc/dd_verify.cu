@@ -214,8 +214,16 @@ __device__ __forceinline__ void fold(Acc& a, const uint4 (&lw)[NV], const uint4 
       a.s1d = __fadd2_rn(a.s1d, ed);
       a.skd = __ffma2_rn(ed, __ffma2_rn(L[k][e], neg1, M[k][e]), a.skd);
     }
-  // --- coupled Gumbel-max samples (same noise for both); best score + its vector
+  // --- coupled Gumbel-max samples (same noise for both); best score + its vector.
+  // Screening: a group of four entries needs its exact noise only if an upper
+  // bound of its scores beats the best exact score any lane of the warp has seen
+  // in this row (all lanes work on one row); otherwise none of its scores can be
+  // the row's maximum, nor tie with it. The bound costs one lg2; candidates get
+  // exactly the fp32 noise and scores they always got.
   if constexpr (SAMPLE) {
+    const unsigned act = __activemask();
+    const float tht = ordered_to_float(__reduce_max_sync(act, float_to_ordered(a.bt)));
+    const float thd = ordered_to_float(__reduce_max_sync(act, float_to_ordered(a.bd)));
     const float2 it2 = make_float2(invT, invT);
 #pragma unroll
     for (int k = 0; k < NV; ++k) {
@@ -224,14 +232,24 @@ __device__ __forceinline__ void fold(Acc& a, const uint4 (&lw)[NV], const uint4 
       for (int q = 0; q < VEC / 4; ++q) {
         const PhiloxOut o = philox4x32_10((uint32_t)(v0[k] >> 2) + q, (uint32_t)pos,
                                           (uint32_t)b, key.step, key.k0, key.k1);
-        const float2 g01 = make_float2(gumbel_from_word(o.w[0]), gumbel_from_word(o.w[1]));
-        const float2 g23 = make_float2(gumbel_from_word(o.w[2]), gumbel_from_word(o.w[3]));
-        const float2 s0 = __ffma2_rn(L[k][2 * q], it2, g01);
-        const float2 s1 = __ffma2_rn(L[k][2 * q + 1], it2, g23);
-        const float2 d0 = __ffma2_rn(M[k][2 * q], it2, g01);
-        const float2 d1 = __ffma2_rn(M[k][2 * q + 1], it2, g23);
-        bt = fmaxf(bt, fmaxf(fmaxf(s0.x, s0.y), fmaxf(s1.x, s1.y)));
-        bd = fmaxf(bd, fmaxf(fmaxf(d0.x, d0.y), fmaxf(d1.x, d1.y)));
+        const float2 u01 = make_float2(gumbel_bound_from_word(o.w[0]), gumbel_bound_from_word(o.w[1]));
+        const float2 u23 = make_float2(gumbel_bound_from_word(o.w[2]), gumbel_bound_from_word(o.w[3]));
+        const float2 s0 = __ffma2_rn(L[k][2 * q], it2, u01);
+        const float2 s1 = __ffma2_rn(L[k][2 * q + 1], it2, u23);
+        const float2 d0 = __ffma2_rn(M[k][2 * q], it2, u01);
+        const float2 d1 = __ffma2_rn(M[k][2 * q + 1], it2, u23);
+        const float ubt = fmaxf(fmaxf(s0.x, s0.y), fmaxf(s1.x, s1.y));
+        const float ubd = fmaxf(fmaxf(d0.x, d0.y), fmaxf(d1.x, d1.y));
+        if (ubt > tht || ubd > thd) {
+          const float2 g01 = make_float2(gumbel_from_word(o.w[0]), gumbel_from_word(o.w[1]));
+          const float2 g23 = make_float2(gumbel_from_word(o.w[2]), gumbel_from_word(o.w[3]));
+          const float2 e0 = __ffma2_rn(L[k][2 * q], it2, g01);
+          const float2 e1 = __ffma2_rn(L[k][2 * q + 1], it2, g23);
+          const float2 f0 = __ffma2_rn(M[k][2 * q], it2, g01);
+          const float2 f1 = __ffma2_rn(M[k][2 * q + 1], it2, g23);
+          bt = fmaxf(bt, fmaxf(fmaxf(e0.x, e0.y), fmaxf(e1.x, e1.y)));
+          bd = fmaxf(bd, fmaxf(fmaxf(f0.x, f0.y), fmaxf(f1.x, f1.y)));
+        }
       }
       if (bt > a.bt) { a.bt = bt; a.vbt = v0[k]; }
       if (bd > a.bd) { a.bd = bd; a.vbd = v0[k]; }
