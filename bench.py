@@ -388,7 +388,7 @@ def run_ours(args, world, rank, local):
                    "l2": "flushed between steps (256 MiB write outside the step's event "
                          "window); the logits (%.0f MB) also exceed L2" % (vbytes / 1e6)},
         "phases_ms": {"attention": a_ms, "verify": v_ms, "select_decide": s_ms},
-        "roofline": {"bound": "hbm", "kernel": "verify_logits_kernel", "achieved": achieved,
+        "roofline": {"bound": "hbm", "kernel": "verify_stream_kernel (+ its row merge; one graph, timed together)", "achieved": achieved,
                      "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                      "traffic": recorded_traffic("dd_verify.cu", spec.name),
                      "algorithmic_bytes": vbytes,
