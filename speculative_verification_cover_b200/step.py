@@ -6,7 +6,7 @@ A step is the four library calls in order, on one stream:
   3. dd_select_seeds        -- the next step's seed set from u, d_in, d_out
   4. dd_decide              -- KEEP / REPLACE / REMASK
 Buffers are allocated once (torch, caller side); the library itself never
-allocates. The three phases can be captured into CUDA graphs and replayed.
+allocates. The step (and each of its three phases) can be captured into CUDA graphs and replayed.
 """
 from __future__ import annotations
 
@@ -94,6 +94,8 @@ class VerifyStep:
 
     # --- CUDA graphs
     def capture(self):
+        """Capture the step as one CUDA graph (what a serving loop replays) and, for the
+        per-phase breakdown, each of the three phases as a graph of its own."""
         self()  # warm every kernel (lazy attribute set-up happens outside capture)
         torch.cuda.synchronize()
         graphs = []
@@ -102,25 +104,30 @@ class VerifyStep:
             with torch.cuda.graph(g):
                 fn()
             graphs.append(g)
+        whole = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(whole):
+            self()
+        graphs.append(whole)
         torch.cuda.synchronize()
         self.graphs = graphs
         return graphs
 
     def replay(self, events=None):
-        """Replay the captured phases; events (4 timing events or None) are recorded
-        before attention, before verify, after verify and at the end."""
-        ga, gv, gs = self.graphs
-        if events:
-            events[0].record()
+        """Replay the step. Without events: the one-graph step. With 4 timing events:
+        the three phase graphs, with the events recorded before attention, before
+        verify, after verify and at the end (the events between phases cost a few
+        microseconds of their own)."""
+        ga, gv, gs, whole = self.graphs
+        if not events:
+            whole.replay()
+            return
+        events[0].record()
         ga.replay()
-        if events:
-            events[1].record()
+        events[1].record()
         gv.replay()
-        if events:
-            events[2].record()
+        events[2].record()
         gs.replay()
-        if events:
-            events[3].record()
+        events[3].record()
 
     def result_tensors(self):
         """What a caller reads back after a step."""
