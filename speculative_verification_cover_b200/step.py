@@ -49,6 +49,7 @@ class VerifyStep:
         self.new_tokens = torch.empty(B, L, dtype=torch.int32, device=dev)
         self.accepted = torch.empty(B, dtype=torch.uint8, device=dev)
         self.graphs = None
+        self.side = None
 
     # --- the four calls
     def attention(self):
@@ -77,6 +78,21 @@ class VerifyStep:
         self.verify()
         self.select_and_decide()
 
+    def forked(self):
+        """The same step with the vocabulary pass on a side stream, concurrent with the
+        attention call (they share no data; selection needs both, so the streams join
+        before it). The attention kernels leave SMs idle at small shapes and the
+        vocabulary pass fills them."""
+        main = torch.cuda.current_stream()
+        if self.side is None:
+            self.side = torch.cuda.Stream(device=main.device)
+        self.side.wait_stream(main)
+        with torch.cuda.stream(self.side):
+            self.verify()
+        self.attention()
+        main.wait_stream(self.side)
+        self.select_and_decide()
+
     def choose_initial_seeds(self):
         """Pass 0 with an empty seed set, then the stability score picks the seeds the
         step will verify (the seeds of step t come from the scores of step t-1)."""
@@ -94,8 +110,9 @@ class VerifyStep:
 
     # --- CUDA graphs
     def capture(self):
-        """Capture the step as one CUDA graph (what a serving loop replays) and, for the
-        per-phase breakdown, each of the three phases as a graph of its own."""
+        """Capture the step as one CUDA graph (what a serving loop replays; the
+        vocabulary pass runs beside the attention call) and, for the per-phase
+        breakdown, each of the three phases as a graph of its own."""
         self()  # warm every kernel (lazy attribute set-up happens outside capture)
         torch.cuda.synchronize()
         graphs = []
@@ -106,7 +123,7 @@ class VerifyStep:
             graphs.append(g)
         whole = torch.cuda.CUDAGraph()
         with torch.cuda.graph(whole):
-            self()
+            self.forked()
         graphs.append(whole)
         torch.cuda.synchronize()
         self.graphs = graphs
