@@ -102,7 +102,6 @@ dd_status dd_dualview_attention(const void* q, const void* k_cur, const void* v_
   a.din_part = reinterpret_cast<float*>(w + ws.din_off);
   a.mrows = reinterpret_cast<int32_t*>(w + ws.mrows_off);
   a.mcount = reinterpret_cast<int32_t*>(w + ws.mcount_off);
-  a.seedbits = reinterpret_cast<uint32_t*>(w + ws.seedbits_off);
   a.newbits = reinterpret_cast<uint32_t*>(w + ws.newbits_off);
   a.mrank = reinterpret_cast<int32_t*>(w + ws.mrank_off);
   a.k_view = w + ws.kview_off;

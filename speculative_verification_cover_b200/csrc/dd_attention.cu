@@ -25,8 +25,7 @@ AttnWorkspace attn_workspace_layout(int B, int L, int Hq, int Hkv, int d) {
   w.mrows_off = up(w.din_off + part);
   w.mcount_off = up(w.mrows_off + (size_t)B * L * sizeof(int32_t));
   const size_t words = (size_t)B * ((L + 31) / 32) * sizeof(uint32_t);
-  w.seedbits_off = up(w.mcount_off + (size_t)B * sizeof(int32_t));
-  w.newbits_off = up(w.seedbits_off + words);
+  w.newbits_off = up(w.mcount_off + (size_t)B * sizeof(int32_t));
   w.mrank_off = up(w.newbits_off + words);
   // tensor-core path: bf16 views and the compacted masked rows for pass 2
   w.Lp = (L + 127) / 128 * 128;
@@ -43,7 +42,7 @@ namespace {
 
 // ---------------------------------------------------------------------------
 // Everything the passes need from the flags, one launch, grid (1 + copy blocks, B):
-//   block 0 of sequence b: the seed / newly-written flags packed 32 to a word, the
+//   block 0 of sequence b: the newly-written flags packed 32 to a word, the
 //     masked query rows in ascending order (stable compaction), their count, and
 //     each row's rank among them (-1 for a row that is not masked);
 //   blocks 1.. (tensor-core path with seeds): the drafting view of K and V --
@@ -53,7 +52,7 @@ struct PrepArgs {
   const uint8_t *is_masked, *is_seed, *is_new;
   int L;
   int32_t *mrows, *mcount, *mrank;  // mrows == nullptr: no compaction
-  uint32_t *seedbits, *newbits;
+  uint32_t* newbits;
   // drafting view (view_units == 0: none); rows of row_units 16-byte units
   const uint4 *k_cur, *v_cur, *k_prev, *v_prev;
   uint4 *k_view, *v_view;
@@ -93,13 +92,9 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(const PrepArgs a) {
   const int W = (L + 31) / 32;
   for (int i0 = threadIdx.x & ~31; i0 < W * 32; i0 += blockDim.x) {
     const int i = i0 + (threadIdx.x & 31);
-    const bool fs = a.is_seed != nullptr && i < L && a.is_seed[(int64_t)b * L + i];
     const bool fn = a.is_new != nullptr && i < L && a.is_new[(int64_t)b * L + i];
-    const uint32_t ws = __ballot_sync(0xffffffffu, fs), wn = __ballot_sync(0xffffffffu, fn);
-    if ((threadIdx.x & 31) == 0) {
-      if (a.seedbits) a.seedbits[(int64_t)b * W + i0 / 32] = ws;
-      if (a.newbits) a.newbits[(int64_t)b * W + i0 / 32] = wn;
-    }
+    const uint32_t wn = __ballot_sync(0xffffffffu, fn);
+    if ((threadIdx.x & 31) == 0 && a.newbits) a.newbits[(int64_t)b * W + i0 / 32] = wn;
   }
   if (a.mrows == nullptr) return;
   __shared__ int warp_sums[32];
@@ -439,7 +434,6 @@ cudaError_t launch_attention(const AttnArgs& a, cudaStream_t stream) {
   pa.mrows = need_din ? a.mrows : nullptr;
   pa.mcount = a.mcount;
   pa.mrank = a.mrank;
-  pa.seedbits = a.seedbits;
   pa.newbits = a.newbits;
   unsigned copy_blocks = 0;
   if (a.dtype == DD_BF16 && a.is_seed != nullptr) {

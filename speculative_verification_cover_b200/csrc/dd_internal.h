@@ -36,7 +36,6 @@ struct AttnArgs {
   float* din_part;      // [B, Hq, L]
   int32_t* mrows;       // [B, L] masked rows of each sequence, ascending
   int32_t* mcount;      // [B]
-  uint32_t* seedbits;   // [B, ceil(L/32)] packed is_seed
   uint32_t* newbits;    // [B, ceil(L/32)] packed is_new
   int32_t* mrank;       // [B, L] rank of a masked row among its sequence's masked rows, else -1
   // tensor-core path only (bf16)
@@ -48,7 +47,7 @@ struct AttnArgs {
 
 // Workspace layout shared by the entry point and the kernels.
 struct AttnWorkspace {
-  size_t dout_off, din_off, mrows_off, mcount_off, seedbits_off, newbits_off, mrank_off;
+  size_t dout_off, din_off, mrows_off, mcount_off, newbits_off, mrank_off;
   size_t kview_off, vview_off, qm_off, lse2m_off, total;
   int Lp;
 };
@@ -80,7 +79,8 @@ cudaError_t launch_selftest_wait(uint32_t limit, cudaStream_t stream);
 
 // Largest L dd_select_seeds handles (keys of one sequence live in shared memory).
 constexpr int kSelectMaxL = 24576;
-// Longest sequence the tensor-core attention handles (packed masks live in shared memory).
+// Longest sequence the tensor-core attention handles (a sequence's packed newly-written
+// flags live in shared memory).
 constexpr int kTcMaxL = 32768;
 constexpr int kSelectMaxK = 1024;
 
