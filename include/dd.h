@@ -116,7 +116,11 @@ dd_status dd_dualview_attention(
     void* workspace, size_t workspace_bytes, void* stream);
 
 /* Bytes of device scratch dd_dualview_attention needs for these sizes
- * (0 on invalid sizes). Pure host function. */
+ * (0 on invalid sizes). Pure host function. Dominant terms: a bf16 copy of K
+ * and V with the seed rows taken from the cache (2*B*L*Hkv*d*2 bytes) and room
+ * for every query row of the second pass (B*L*Hq*d*2 bytes: how many rows are
+ * still masked is only known on the device), plus per-head fp32 partials of
+ * the statistics (2*B*Hq*L*4 bytes). */
 size_t dd_dualview_attention_workspace_size(int B, int L, int Hq, int Hkv, int d);
 
 /* Per-row outputs of dd_verify_logits, each [B*R] (row-major [B,R]).
