@@ -50,6 +50,19 @@ def test_workspace_size_is_host_only(lib):
     assert dd.dd_dualview_attention_workspace_size(0, 2048, 28, 4, 128) == 0
 
 
+@pytest.mark.parametrize("B,L,Hq,Hkv,d", [(1, 512, 32, 32, 128), (8, 2048, 28, 4, 128),
+                                          (2, 333, 80, 8, 128), (1, 1, 1, 1, 64)])
+def test_attention_workspace_holds_the_documented_terms(lib, B, L, Hq, Hkv, d):
+    # the header's dominant terms: the drafting view of K and V, room for every query
+    # row of pass 2, per-head fp32 partials of d_in / d_out; the rest is per-position
+    # bookkeeping (row lists, ranks, packed flags, lse of the masked rows) and padding
+    n = dd.dd_dualview_attention_workspace_size(B, L, Hq, Hkv, d)
+    dominant = 2 * B * L * Hkv * d * 2 + B * L * Hq * d * 2 + 2 * B * Hq * L * 4
+    lp = (L + 127) // 128 * 128
+    small = B * L * 4 * 2 + B * 4 + B * ((L + 31) // 32) * 4 + B * Hq * lp * 4
+    assert dominant <= n <= dominant + small + 16 * 256
+
+
 P = ctypes.c_void_p
 FAKE = P(0x10000)      # never dereferenced: validation fails first
 MISALIGNED = P(0x10008)
