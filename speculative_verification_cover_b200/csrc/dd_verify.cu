@@ -5,7 +5,9 @@
 // verified row produces: LSE of both, argmax of both, the verifier's max
 // probability, its entropy (the uncertainty u of COVER's seed score),
 // KL(drafter || verifier), and at T > 0 the coupled Gumbel-max samples of both
-// with the same Philox noise.
+// with the same Philox noise (every entry's noise word is drawn, but its exact
+// Gumbel value is computed only where a cheap upper bound says the entry could
+// still be the row's maximum; see fold()).
 //
 // Work decomposition: the 16-byte vectors of all rows form one index space
 // (rows x vectors per row); it is split into equal contiguous ranges, one per
