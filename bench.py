@@ -201,6 +201,23 @@ def recorded_traffic(kernel_file, workload_name):
     return None
 
 
+# Attention layers of the models the workloads are shaped like. These are model
+# facts, not on the pages: the multi-layer figure built from them is a projection.
+MODEL_LAYERS = {"llada8b": 32, "dream7b": 28, "sdar8b": 36}
+
+
+def projection(spec_name, a_ms, v_ms, s_ms):
+    """A whole-model verification step from the measured phases: one attention call per
+    layer, one vocabulary pass and one selection + decision per step (phases in series)."""
+    layers = MODEL_LAYERS.get(spec_name.split("_")[0])
+    if layers is None:
+        return None
+    ms = layers * a_ms + v_ms + s_ms
+    return {"layers": layers, "ms_per_step": ms, "steps_per_s": 1000.0 / ms,
+            "note": "projection: layer count assumed (model fact, not on the pages); "
+                    "phases of the per-phase pass composed in series"}
+
+
 # ----------------------------------------------------------------------------- CPU oracle
 def oracle_step(x, spec, b, head_stride=1, row_stride=1, seed=2024, step_index=1):
     """One verification step of sequence b on the CPU oracle (optionally a sample:
@@ -397,6 +414,7 @@ def run_ours(args, world, rank, local):
         "vs_baseline": None, "dtype": "bf16" if spec.dtype == "bf16" else "f32",
         "data": "synthetic (seeded; shapes and distributions of the named model)",
         "positions_per_s": value * spec.B * spec.R,
+        "attention_tokens_per_s": value * spec.B * spec.L,
         "config": {"workload": spec.name, "B": spec.B, "L": spec.L, "Hq": spec.Hq,
                    "Hkv": spec.Hkv, "d": spec.d, "V": spec.V, "R": spec.R, "seeds": spec.k,
                    "temperature": spec.temperature, "policy": spec.policy,
@@ -407,6 +425,7 @@ def run_ours(args, world, rank, local):
                          "window); the logits (%.0f MB) also exceed L2" % (vbytes / 1e6)},
         "phases_ms": {"attention": a_ms, "verify": v_ms, "select_decide": s_ms,
                       "method": "separate pass: three phase graphs, events between them"},
+        "projection": projection(spec.name, a_ms, v_ms, s_ms),
         "roofline": {"bound": "hbm", "kernel": "verify_stream_kernel (+ its row merge; one graph, timed together)", "achieved": achieved,
                      "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                      "traffic": recorded_traffic("dd_verify.cu", spec.name),
