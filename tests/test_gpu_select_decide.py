@@ -4,6 +4,7 @@ import pytest
 import torch
 
 from speculative_verification_cover_b200 import dd
+from oracle import seeds as OS
 from tests import parity as PA
 
 pytestmark = pytest.mark.gpu
@@ -39,38 +40,40 @@ def test_select_matches_oracle(B, L, R, off, k, quant):
     elig = (rng.random((B, L)) < 0.6).astype(np.uint8)
     t = lambda a, dt=torch.float32: torch.tensor(a, dtype=dt, device="cuda")
     seeds, is_seed, score = _select(t(entropy), t(d_in), t(d_out), t(elig, torch.uint8), k, off)
-    ties = 0
+    near = 0
     for b in range(B):
         u = np.zeros(L)
         u[off:off + R] = entropy[b]
         el = elig[b].astype(bool).copy()
         el[:off] = False
         el[off + R:] = False
-        # the GPU computes the score in fp32: feed the oracle the same fp32 inputs
-        u32 = np.float32(u).astype(np.float64)
+        u32, din32, dout32 = (np.float32(a) for a in (u, d_in[b], d_out[b]))
+        # the oracle's fp64 score on the very fp32 inputs the kernel received
         want_seeds, want_is, want_score, margin = PA.oracle_select(
-            u32, np.float32(d_in[b]).astype(np.float64), np.float32(d_out[b]).astype(np.float64),
-            el, k)
-        PA.assert_close("score", np.where(el, PA.np64(score[b]), 0), np.where(el, want_score, 0),
+            u32.astype(np.float64), din32.astype(np.float64), dout32.astype(np.float64), el, k)
+        got_score = PA.np64(score[b])
+        PA.assert_close("score", np.where(el, got_score, 0), np.where(el, want_score, 0),
                         1e-6, 1e-6)
+        assert np.all(np.isneginf(got_score[~el])), b
+        # The set is an integer decided by floating point: both sides decide it in the
+        # kernel's precision. The kernel's fp32 score is u * (1 + d_in) / (1 + d_out)
+        # with IEEE rounding at each operation; numpy's float32 arithmetic in the same
+        # order gives the same bits, and the oracle's rule (score descending, position
+        # ascending) picks the set from them. No sequence is excluded.
+        s32 = (u32 * (np.float32(1) + din32)) / (np.float32(1) + dout32)
+        assert np.array_equal(got_score[el], s32[el].astype(np.float64)), b
+        k_seeds, k_is = OS.select(np.where(el, s32.astype(np.float64), -np.inf), k)
+        assert np.array_equal(PA.npi(seeds[b]), k_seeds), b
+        assert np.array_equal(PA.npi(is_seed[b]), k_is.astype(np.int64)), b
+        # Against the fp64 decision: identical unless the k-th place is a near-tie.
         if margin < PA.TIE_EPS:
-            ties += 1
-            continue
-        # the chosen set is unique away from a tie at the k-th place
-        assert np.array_equal(PA.npi(is_seed[b]), want_is), b
-        got = PA.npi(seeds[b])
-        assert sorted(got[got >= 0]) == sorted(want_seeds[want_seeds >= 0]), b
-        assert np.array_equal(got < 0, want_seeds < 0), b
-        # rank order: descending score, ties (within fp32 rounding) to the lower position
-        chosen = got[got >= 0]
-        for r in range(len(chosen) - 1):
-            sa, sb = want_score[chosen[r]], want_score[chosen[r + 1]]
-            assert sa > sb - PA.TIE_EPS, (b, r)
-            if abs(sa - sb) >= PA.TIE_EPS:
-                assert sa > sb
-            elif sa == sb:
-                assert chosen[r] < chosen[r + 1]
-    assert ties <= B
+            near += 1
+        else:
+            assert np.array_equal(PA.npi(is_seed[b]), want_is), b
+            assert np.array_equal(PA.npi(seeds[b]), want_seeds), b
+    # near-ties at the k-th place are counted; random continuous scores have none
+    assert near == 0 or quant, near
+    assert near <= B
 
 
 POLICIES = ["trust", "kl", "conf", "cover", "coupled"]
@@ -115,10 +118,12 @@ def test_decide_matches_oracle(policy, T):
                 for k, v in stats_np.items()}
         rows["margin_t"] = np.full(R, np.inf)
         rows["margin_d"] = np.full(R, np.inf)
+        # The kernel compares fp32 statistics with fp32 thresholds; the oracle takes
+        # the same decisions on the same values (thresholds rounded to fp32 too), so
+        # every position must agree, near-ties included.
         wd, wt, wa, near = PA.oracle_decide(policy, tokens[b], is_seed[b], elig[b], rows, off, R,
-                                            T, 0.5, 0.6)
-        ok = ~near
-        assert np.array_equal(PA.npi(dec[b])[ok], wd[ok].astype(np.int64)), (policy, b)
-        assert np.array_equal(PA.npi(newt[b])[ok], wt[ok].astype(np.int64)), (policy, b)
-        if not near.any():
-            assert int(acc[b]) == wa
+                                            T, float(np.float32(0.5)), float(np.float32(0.6)))
+        assert np.array_equal(PA.npi(dec[b]), wd.astype(np.int64)), (policy, b)
+        assert np.array_equal(PA.npi(newt[b]), wt.astype(np.int64)), (policy, b)
+        assert int(acc[b]) == wa, (policy, b)
+        assert int(near.sum()) <= 2  # positions within 1e-4 of a threshold: counted

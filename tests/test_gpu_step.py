@@ -51,10 +51,18 @@ def test_tiny_step(T, policy):
     near_rows = PA.compare_verify(stats, ws_, rows, T)
     u = np.zeros(L)
     u[off:] = ws_["entropy_t"]
-    want_seeds, want_is, _, margin = PA.oracle_select(u, wdin, wdout, PA.npi(x["eligible"][0]),
-                                                      spec.k)
-    if margin >= 1e-3:  # GPU scores come from GPU statistics: allow their tolerance
-        assert np.array_equal(PA.npi(next_seed[0]), want_is)
+    elig = PA.npi(x["eligible"][0])
+    want_seeds, want_is, want_score, _ = PA.oracle_select(u, wdin, wdout, elig, spec.k)
+    # The GPU's scores come from the GPU's statistics (entropy, d_in, d_out, each within
+    # its tolerance), so its set may differ from the oracle's only by positions whose
+    # oracle score lies within that tolerance of the k-th boundary.
+    got_is = PA.npi(next_seed[0]).astype(bool)
+    fin = np.sort(want_score[np.isfinite(want_score)])[::-1]
+    mid = 0.5 * (fin[spec.k - 1] + fin[spec.k])
+    band = 4e-3 * (1.0 + abs(mid))
+    diff = got_is != want_is.astype(bool)
+    assert np.all(np.abs(want_score[diff] - mid) <= band), np.nonzero(diff)
+    assert int(diff.sum()) <= 2
     wd, wt, wa, near = PA.oracle_decide(policy, PA.npi(x["tokens"][0]), PA.npi(x["is_seed"][0]),
                                         PA.npi(x["eligible"][0]), ws_, off, R, T, spec.tau_kl,
                                         spec.tau_conf)

@@ -132,3 +132,64 @@ def test_score_formula_swap_is_caught(monkeypatch):
         np.asarray(el).astype(bool), np.asarray(u, float) * (1 + np.asarray(do, float))
         / (1 + np.asarray(di, float)), -np.inf))
     assert _fails(TS.test_stability_score_golden)
+
+
+# --------------------------------------------------------------------- near-tie margins
+from tests import test_oracle_margins as TM  # noqa: E402
+
+
+def test_top2_gap_to_third_entry_is_caught(monkeypatch):
+    def bad(x):  # bug: gap to the third largest entry instead of the runner-up
+        if x.shape[-1] < 3:
+            return np.full(x.shape[:-1], np.inf)
+        part = -np.sort(-x, axis=-1)
+        return part[..., 0] - part[..., 2]
+
+    monkeypatch.setattr(vb, "_top2_gap", bad)
+    assert _fails(TM.test_top2_gap_special_cases)
+    assert _fails(TM.test_top2_gap_matches_pairwise_brute_force, 1)
+
+
+def test_top2_gap_of_logits_instead_of_scores_is_caught(monkeypatch):
+    orig = vb.coupled_samples
+
+    def bad(l, m, temperature, g):  # bug: margins of the raw logits, not of l/T + g
+        out = orig(l, m, temperature, g)
+        out["margin_t"] = vb._top2_gap(np.asarray(l, dtype=np.float64))
+        out["margin_d"] = vb._top2_gap(np.asarray(m, dtype=np.float64))
+        return out
+
+    monkeypatch.setattr(vb, "coupled_samples", bad)
+    assert _fails(TM.test_coupled_margins_are_gaps_of_the_noisy_scores)
+
+
+def test_top2_gap_absolute_value_hides_ties_is_caught(monkeypatch):
+    # bug: a zero gap (tied leaders) reported as the gap to the next distinct value
+    def bad(x):
+        out = []
+        for r in np.asarray(x).reshape(-1, np.asarray(x).shape[-1]):
+            u = np.unique(r)[::-1]
+            out.append(u[0] - u[1] if len(u) > 1 else np.inf)
+        return np.array(out).reshape(np.asarray(x).shape[:-1])
+
+    monkeypatch.setattr(vb, "_top2_gap", bad)
+    assert _fails(TM.test_top2_gap_special_cases)
+
+
+def test_boundary_margin_off_by_one_is_caught(monkeypatch):
+    def bad(score, k):  # bug: compares the (k+1)-th and (k+2)-th scores
+        s = np.sort(np.asarray(score, dtype=np.float64)[np.isfinite(score)])[::-1]
+        if len(s) <= k + 1 or k == 0:
+            return np.inf
+        return s[k] - s[k + 1]
+
+    monkeypatch.setattr(sd, "boundary_margin", bad)
+    assert _fails(TM.test_boundary_margin_special_cases)
+    assert _fails(TM.test_boundary_margin_is_the_selection_stability_margin, 0)
+
+
+def test_boundary_margin_always_zero_is_caught(monkeypatch):
+    # a margin that skipped every sequence would make the GPU seed tests vacuous
+    monkeypatch.setattr(sd, "boundary_margin", lambda score, k: 0.0)
+    assert _fails(TM.test_boundary_margin_special_cases)
+    assert _fails(TM.test_boundary_margin_matches_brute_force, 3)
