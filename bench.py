@@ -18,7 +18,11 @@ Rank 0 prints one JSON line:
   roofline  the dominant kernel (the vocabulary pass: HBM-bound) against the
             measured HBM copy bandwidth; attention is reported beside it
             against the measured dense bf16 tensor peak
-  cpu_baseline  the fp64 CPU oracle on a bounded sample (rank 0, N = 1 only)
+  cpu_baseline  the fp64 CPU oracle on a bounded sample (rank 0, N = 1 only),
+            with the oracle's near-tie counts (positions within 1e-4 of a tie or
+            a threshold) on that sample
+  workloads the other four workloads (N = 1 only; --no-workloads skips them),
+            each a few steps: throughput, both rooflines, clocks, near-tie counts
 Under torchrun (N > 1) each rank runs its own batch (weak scaling, no
 collective on the data path; the only collectives are the timing barrier and
 max-reduce).
@@ -26,7 +30,6 @@ max-reduce).
 from __future__ import annotations
 
 import argparse
-import hashlib
 import json
 import math
 import os
@@ -58,6 +61,8 @@ def parse():
     p.add_argument("--impl", choices=("ours", "reference"), default="ours")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    p.add_argument("--no-workloads", action="store_true",
+                   help="skip the per-workload block (the other four workloads, N = 1 only)")
     return p.parse_args()
 
 
@@ -180,49 +185,23 @@ def algorithmic(spec):
     return verify_bytes, attn_flops, pass2_flops
 
 
-def recorded_traffic(kernel_file, workload_name):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on this
-    workload and on the current source of the kernel (both recorded beside the figure)."""
-    src = os.path.join(ROOT, "speculative_verification_cover_b200", "csrc", kernel_file)
-    summ = os.path.join(ROOT, "profiles", "verify_logits_%s.md" % workload_name.split("_")[0])
-    if not (os.path.exists(src) and os.path.exists(summ)):
-        return None
-    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    rec = {}
-    for line in open(summ):
-        if line.startswith("traffic_bytes_per_launch:"):
-            rec["bytes"] = float(line.split(":", 1)[1])
-        if line.startswith("source_sha256_16:"):
-            rec["sha"] = line.split(":", 1)[1].strip()
-        if line.startswith("workload:"):
-            rec["workload"] = line.split(":", 1)[1].strip()
-    if rec.get("sha") == h and rec.get("workload") == workload_name and "bytes" in rec:
-        return rec["bytes"]
-    return None
-
-
-# Attention layers of the models the workloads are shaped like. These are model
-# facts, not on the pages: the multi-layer figure built from them is a projection.
-MODEL_LAYERS = {"llada8b": 32, "dream7b": 28, "sdar8b": 36}
-
-
-def projection(spec_name, a_ms, v_ms, s_ms):
-    """A whole-model verification step from the measured phases: one attention call per
-    layer, one vocabulary pass and one selection + decision per step (phases in series)."""
-    layers = MODEL_LAYERS.get(spec_name.split("_")[0])
-    if layers is None:
-        return None
-    ms = layers * a_ms + v_ms + s_ms
-    return {"layers": layers, "ms_per_step": ms, "steps_per_s": 1000.0 / ms,
-            "note": "projection: layer count assumed (model fact, not on the pages); "
-                    "phases of the per-phase pass composed in series"}
+def recorded_traffic(workload_name):
+    """DRAM bytes per launch of the vocabulary kernel on this workload, from the
+    machine-written ncu record (profiles/traffic.json), if it was taken on the
+    current source of the kernel; else None."""
+    from speculative_verification_cover_b200 import profiling
+    return profiling.lookup("verify_stream_kernel", workload_name)
 
 
 # ----------------------------------------------------------------------------- CPU oracle
-def oracle_step(x, spec, b, head_stride=1, row_stride=1, seed=2024, step_index=1):
+def oracle_step(x, spec, b, head_stride=1, row_stride=1, seed=2024, step_index=1, near=None):
     """One verification step of sequence b on the CPU oracle (optionally a sample:
     every head_stride-th head and every row_stride-th verified row). Returns seconds
-    per full step, extrapolated from the sample."""
+    per full step, extrapolated from the sample. With `near` (a dict), also counts
+    what the oracle puts within 1e-4 of a tie or a threshold: sampled rows whose
+    coupled sample leads its runner-up by less (rows), decided positions whose
+    statistic lies that close to the policy's threshold or tie (decisions), and
+    whether the seed set's k-th place is that close (seed_boundary)."""
     from oracle import attention as OA
     from oracle import decide as OD
     from oracle import seeds as OS
@@ -249,11 +228,45 @@ def oracle_step(x, spec, b, head_stride=1, row_stride=1, seed=2024, step_index=1
     full = {k: np.zeros(spec.R, dtype=v.dtype) for k, v in st.items()}
     for k, v in st.items():
         full[k][rows] = v
-    OD.decide(spec.policy, x["tokens"][b].cpu().numpy(), seeds, x["eligible"][b].cpu().numpy(),
-              full, spec.pos_offset, spec.R, spec.temperature, spec.tau_kl, spec.tau_conf)
+    dec, _, _, near_dec = OD.decide(spec.policy, x["tokens"][b].cpu().numpy(), seeds,
+                                    x["eligible"][b].cpu().numpy(), full, spec.pos_offset,
+                                    spec.R, spec.temperature, spec.tau_kl, spec.tau_conf)
     t3 = time.perf_counter()
+    if near is not None:
+        sampled_pos = np.zeros(spec.L, dtype=bool)
+        sampled_pos[spec.pos_offset + rows] = True
+        near["rows"] = near.get("rows", 0) + len(rows)
+        near["near_rows"] = near.get("near_rows", 0) + int(
+            ((st["margin_t"] < 1e-4) | (st["margin_d"] < 1e-4)).sum())
+        near["decisions"] = near.get("decisions", 0) + int(((dec > 0) & sampled_pos).sum())
+        near["near_decisions"] = near.get("near_decisions", 0) + int((near_dec & sampled_pos).sum())
+        if head_stride == 1 and row_stride == 1 and spec.k > 0:
+            near["seed_boundary_near"] = near.get("seed_boundary_near", 0) + int(
+                OS.boundary_margin(score, spec.k) < 1e-4)
     per_seq = ((t1 - t0) * spec.Hq / len(heads) + (t2 - t1) * spec.R / len(rows) + (t3 - t2))
     return per_seq * spec.B
+
+
+def oracle_near_ties(x, spec, nrows=32):
+    """Near-tie counts of the oracle on a bounded sample of a workload: nrows evenly
+    spaced verified rows of sequence 0 (vocabulary statistics and decisions only; the
+    attention statistics are not sampled here)."""
+    from oracle import decide as OD
+    from oracle import vocab as OV
+    f64 = lambda t: t.detach().float().cpu().numpy().astype(np.float64)
+    rows = np.unique(np.linspace(0, spec.R - 1, min(nrows, spec.R)).astype(np.int64))
+    idx = torch.as_tensor(rows, device=x["logits_t"].device)
+    st = OV.verify_rows(f64(x["logits_t"][0][idx]), f64(x["logits_d"][0][idx]),
+                        spec.temperature, 2024, 1, 0, rows + spec.pos_offset)
+    pos = rows + spec.pos_offset
+    dec, _, _, near_dec = OD.decide(
+        spec.policy, x["tokens"][0].cpu().numpy()[pos], x["is_seed"][0].cpu().numpy()[pos],
+        x["eligible"][0].cpu().numpy()[pos], st, 0, len(rows), spec.temperature, spec.tau_kl,
+        spec.tau_conf)
+    return {"rows": int(len(rows)),
+            "near_rows": int(((st["margin_t"] < 1e-4) | (st["margin_d"] < 1e-4)).sum()),
+            "decisions": int((dec > 0).sum()), "near_decisions": int(near_dec.sum()),
+            "sample": f"{len(rows)} evenly spaced verified rows of sequence 0"}
 
 
 def blas_threads():
@@ -268,15 +281,19 @@ def blas_threads():
 def cpu_baseline(x, spec, budget_s=12.0):
     """Full oracle steps of sequence 0 until ~budget_s of host time."""
     per, n, t0 = [], 0, time.perf_counter()
+    near = {}
     while n == 0 or (time.perf_counter() - t0) < budget_s:
-        per.append(oracle_step(x, spec, b=n % spec.B))
+        per.append(oracle_step(x, spec, b=n % spec.B, near=near if n < spec.B else None))
         n += 1
         if n >= 20:
             break
     sec = float(np.mean(per))
+    near["sample"] = (f"the oracle's own statistics of the first {min(n, spec.B)} full "
+                      "step(s) above: positions within 1e-4 of a tie or a threshold")
     return {"value": 1.0 / sec, "unit": "steps/s", "cores": blas_threads(), "kind": "oracle",
             "sample": f"{n} full fp64 oracle step(s) of one sequence of {spec.name} "
-                      f"(all {spec.Hq} heads, all {spec.R} rows), scaled to the batch of {spec.B}"}
+                      f"(all {spec.Hq} heads, all {spec.R} rows), scaled to the batch of {spec.B}",
+            "near_ties": near}
 
 
 # ----------------------------------------------------------------------------- arms
@@ -352,24 +369,20 @@ def run_e2e(step, x, K, world):
             "d2h_bytes_per_step": d2h}
 
 
-def run_ours(args, world, rank, local):
+def measure(spec, dev, K, warmup, world, rank, flush):
+    """Inputs, the step graph, W warm-up and K timed steps of one workload. Returns the
+    inputs, the step and the timings (max over ranks)."""
     from speculative_verification_cover_b200 import dd
-    from speculative_verification_cover_b200.step import INPUT_KEYS, KERNELS_PER_STEP, VerifyStep
-    dd.lib()  # fail loudly if the library is missing
-    spec = spec_by_name(args.workload, args.batch)
-    dev = torch.device("cuda", local)
+    from speculative_verification_cover_b200.step import VerifyStep
     x = W.make_inputs(spec, dev, seed=shard_seed(spec, rank))
     step = VerifyStep(spec, x)
     step.choose_initial_seeds()
     step.capture()
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    for _ in range(max(args.warmup, 3)):
+    for _ in range(max(warmup, 3)):
         flush.zero_()
         step.replay()
     torch.cuda.synchronize()
     assert dd.dd_get_device_error() == dd.DD_OK
-
-    K = args.steps
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(K)]
     with ClockSampler(dev.index) as clocks:
@@ -401,20 +414,83 @@ def run_ours(args, world, rank, local):
     ms, a_ms, v_ms, s_ms = max_over_ranks([mean(step_ms), mean(attn_ms), mean(ver_ms),
                                            mean(sel_ms)], world)
     assert dd.dd_get_device_error() == dd.DD_OK
+    return x, step, dict(ms=ms, a_ms=a_ms, v_ms=v_ms, s_ms=s_ms, clocks=clocks.summary())
+
+
+def derived(spec, t, world):
+    """Throughput and roofline figures of one workload's timings."""
+    hbm, bf16, _, peak_src = peaks()
+    vbytes, aflops, pflops = algorithmic(spec)
+    value = world * 1000.0 / t["ms"]
+    gbs = vbytes / (t["v_ms"] * 1e-3) / 1e9
+    tflops = (aflops + pflops) / (t["a_ms"] * 1e-3) / 1e12
+    return {
+        "steps_per_s": value, "ms_per_step": t["ms"],
+        "positions_per_s": value * spec.B * spec.R,
+        "attention_tokens_per_s": value * spec.B * spec.L,
+        "phases_ms": {"attention": t["a_ms"], "verify": t["v_ms"], "select_decide": t["s_ms"],
+                      "method": "separate pass: three phase graphs, events between them"},
+        "verify": {"bound": "hbm", "achieved_gbs": gbs, "peak_gbs": hbm, "frac": gbs / hbm,
+                   "algorithmic_bytes": vbytes, "traffic": recorded_traffic(spec.name),
+                   "peak_source": f"MEASURED_PEAKS.json hbm_gbs ({peak_src})"},
+        "attention": {"bound": "tensor", "algorithmic_flop": aflops + pflops,
+                      "achieved_tflops": tflops, "peak_tflops": bf16, "frac": tflops / bf16,
+                      "peak_source": f"MEASURED_PEAKS.json bf16_tflops ({peak_src})"},
+        "clocks": t["clocks"],
+    }
+
+
+def run_workloads_block(args, dev, flush, with_oracle):
+    """The other four workloads at N = 1, each for a few steps: throughput, both
+    rooflines, clocks, and (from the CPU-baseline leg) the oracle's near-tie counts on
+    a bounded sample."""
+    from speculative_verification_cover_b200 import dd
+    out = []
+    for spec in W.WORKLOADS:
+        if spec.name == args.workload:
+            continue
+        K = max(3, min(args.steps, 20))
+        x, step, t = measure(spec, dev, K, 3, 1, 0, flush)
+        e = {"workload": spec.name, "steps": K, "warmup": 3,
+             "dtype": "bf16" if spec.dtype == "bf16" else "f32",
+             "config": {"B": spec.B, "L": spec.L, "Hq": spec.Hq, "Hkv": spec.Hkv, "d": spec.d,
+                        "V": spec.V, "R": spec.R, "seeds": spec.k,
+                        "temperature": spec.temperature, "policy": spec.policy},
+             "gpu_launches": 0}
+        e.update(derived(spec, t, 1))
+        if with_oracle:
+            e["oracle_near_ties"] = oracle_near_ties(x, spec)
+        out.append(e)
+        step.graphs = None
+        del x, step
+        torch.cuda.empty_cache()
+        assert dd.dd_get_device_error() == dd.DD_OK
+    return out
+
+
+def run_ours(args, world, rank, local):
+    from speculative_verification_cover_b200 import dd
+    from speculative_verification_cover_b200.step import KERNELS_PER_STEP
+    dd.lib()  # fail loudly if the library is missing
+    spec = spec_by_name(args.workload, args.batch)
+    dev = torch.device("cuda", local)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    K = args.steps
+    x, step, t = measure(spec, dev, K, args.warmup, world, rank, flush)
 
     # ---- end to end through the public API: pinned host inputs -> device -> host decisions
     e2e = None if args.no_e2e else run_e2e(step, x, K, world)
-    hbm, bf16, bf16_s, peak_src = peaks()
-    vbytes, aflops, pflops = algorithmic(spec)
-    achieved = vbytes / (v_ms * 1e-3) / 1e9
-    value = world * 1000.0 / ms
+    d = derived(spec, t, world)
+    value = d["steps_per_s"]
+    ver = d["verify"]
     line = {
         "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world, "steps": K,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16" if spec.dtype == "bf16" else "f32",
+        "warmup": args.warmup, "ms_per_step": t["ms"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if spec.dtype == "bf16" else "f32",
         "data": "synthetic (seeded; shapes and distributions of the named model)",
-        "positions_per_s": value * spec.B * spec.R,
-        "attention_tokens_per_s": value * spec.B * spec.L,
+        "positions_per_s": d["positions_per_s"],
+        "attention_tokens_per_s": d["attention_tokens_per_s"],
         "config": {"workload": spec.name, "B": spec.B, "L": spec.L, "Hq": spec.Hq,
                    "Hkv": spec.Hkv, "d": spec.d, "V": spec.V, "R": spec.R, "seeds": spec.k,
                    "temperature": spec.temperature, "policy": spec.policy,
@@ -422,28 +498,30 @@ def run_ours(args, world, rank, local):
                    "parallelism": f"{world} replica(s), independent batches" if world > 1
                    else "1 GPU",
                    "l2": "flushed between steps (256 MiB write outside the step's event "
-                         "window); the logits (%.0f MB) also exceed L2" % (vbytes / 1e6)},
-        "phases_ms": {"attention": a_ms, "verify": v_ms, "select_decide": s_ms,
-                      "method": "separate pass: three phase graphs, events between them"},
-        "projection": projection(spec.name, a_ms, v_ms, s_ms),
-        "roofline": {"bound": "hbm", "kernel": "verify_stream_kernel (+ its row merge; one graph, timed together)", "achieved": achieved,
-                     "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                     "traffic": recorded_traffic("dd_verify.cu", spec.name),
-                     "algorithmic_bytes": vbytes,
-                     "peak_source": f"MEASURED_PEAKS.json hbm_gbs ({peak_src})"},
-        "attention": {"bound": "tensor", "algorithmic_flop": aflops + pflops,
-                      "achieved_tflops": (aflops + pflops) / (a_ms * 1e-3) / 1e12,
-                      "peak_tflops": bf16, "frac": (aflops + pflops) / (a_ms * 1e-3) / 1e12 / bf16,
-                      "peak_source": f"MEASURED_PEAKS.json bf16_tflops ({peak_src})"},
+                         "window); the logits (%.0f MB) also exceed L2"
+                         % (ver["algorithmic_bytes"] / 1e6)},
+        "phases_ms": d["phases_ms"],
+        "roofline": {"bound": "hbm",
+                     "kernel": "verify_stream_kernel (+ its row merge; one graph, timed together)",
+                     "achieved": ver["achieved_gbs"], "peak": ver["peak_gbs"], "unit": "GB/s",
+                     "frac": ver["frac"], "traffic": ver["traffic"],
+                     "algorithmic_bytes": ver["algorithmic_bytes"],
+                     "peak_source": ver["peak_source"]},
+        "attention": d["attention"],
         "e2e": e2e,
         "gpu_launches": KERNELS_PER_STEP * K,
-        "clocks": clocks.summary(),
+        "clocks": t["clocks"],
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    with_oracle = rank == 0 and world == 1 and not args.no_cpu_baseline
+    if with_oracle:
         line["cpu_baseline"] = cpu_baseline(x, spec)
+    step.graphs = None  # release graphs before the process group
+    del x, step
+    torch.cuda.empty_cache()
+    if world == 1 and not args.no_workloads:
+        line["workloads"] = run_workloads_block(args, dev, flush, with_oracle)
     if rank == 0:
         print(json.dumps(line), flush=True)
-    step.graphs = None  # release graphs before the process group
 
 
 def main():

@@ -283,6 +283,25 @@ uint32_t dd_set_spin_limit(uint32_t limit);
  */
 dd_status dd_selftest_bounded_wait(uint32_t spin_limit, void* stream);
 
+/*
+ * dd_selftest_gumbel_screen -- self-test of the screen dd_verify_logits uses to
+ * skip the exact Gumbel noise of entries that cannot be sampled ([SPOT]
+ * Coupled-Noise Verification; the screen itself is this library's, the pages
+ * have no counterpart). For every noise level k = word >> 9 (2^23 levels) it
+ * writes the library's fp32 noise g_of_level[k] = -ln(-ln U) and the screen's
+ * exact-float j_of_level[k] = 2^23 - 1 - k; for each of the n requested levels
+ * G = g_req[i] it writes limit[i], the screen's bound: a word is screened out at
+ * level G iff its j + 1/2 >= limit. The screen is sound iff every level with
+ * g_of_level[k] > G has j + 1/2 < limit. *gumbel_max (host pointer, may be NULL)
+ * receives the constant above which a required level skips the noise entirely;
+ * sound iff no g_of_level exceeds it.
+ * g_of_level, j_of_level  device, 2^23 floats each
+ * g_req, limit            device, n floats each (may be NULL when n == 0)
+ * Errors: DD_ERR_INVALID_ARG for NULL buffers or n < 0.
+ */
+dd_status dd_selftest_gumbel_screen(float* g_of_level, float* j_of_level, const float* g_req,
+                                    float* limit, int n, float* gumbel_max, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

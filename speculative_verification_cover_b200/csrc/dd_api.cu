@@ -223,4 +223,13 @@ dd_status dd_selftest_bounded_wait(uint32_t limit, void* stream) {
   return from_cuda(launch_selftest_wait(limit, static_cast<cudaStream_t>(stream)));
 }
 
+dd_status dd_selftest_gumbel_screen(float* g_of_level, float* j_of_level, const float* g_req,
+                                    float* limit, int n, float* gumbel_max, void* stream) {
+  if (!g_of_level || !j_of_level || n < 0 || (n > 0 && (!g_req || !limit)))
+    return DD_ERR_INVALID_ARG;
+  if (gumbel_max) *gumbel_max = gumbel_max_constant();
+  return from_cuda(launch_selftest_gumbel(g_of_level, j_of_level, g_req, limit, n,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

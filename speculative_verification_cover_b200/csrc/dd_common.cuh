@@ -70,6 +70,12 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t phase,
   return false;
 }
 
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // ---------------------------------------------------------------------------
 // Philox4x32-10 (Salmon, Moraes, Dror, Shaw, SC'11): ten rounds of
 //   (x0,x1,x2,x3) -> (hi(M1*x2)^x1^k0, lo(M1*x2), hi(M0*x0)^x3^k1, lo(M0*x0))
@@ -107,16 +113,84 @@ __device__ __forceinline__ float gumbel_from_word(uint32_t w) {
   return -__logf(e);
 }
 
-// An upper bound of gumbel_from_word(w) as computed above (its fp32 result),
-// cheap enough to screen every entry: -ln(-ln U) <= -ln(1 - U) since
-// -ln U >= 1 - U on (0, 1). With k = w >> 9, 1 - U = (j + 1/2) 2^-23 exactly for
-// j = 2^23 - 1 - k, so -ln(1 - U) = ln2 (23 - log2(j + 1/2)); j + 1/2 is formed
-// exactly from the float with bits (2^23 + j) minus (2^23 - 1/2). The 0.01
-// margin covers the approximate log2 here (about 4e-6 absolute) and the fp32
-// rounding of the exact path (about 1e-5): the bound is never below it.
-__device__ __forceinline__ float gumbel_bound_from_word(uint32_t w) {
-  const float jh = __uint_as_float((w >> 9) ^ 0x4B7FFFFFu) - 8388607.5f;
-  return fmaf(__log2f(jh), -0.69314718f, 23.f * 0.69314718f + 0.01f);
+// ---------------------------------------------------------------------------
+// Philox4x32-10 split for a streaming pass over one row. In the counter
+// (c0 = v >> 2, c1 = pos, c2 = b, c3 = step) only c0 changes along a row, and
+// rounds 1 and 2 of the generator combine it with the fixed words in a way that
+// leaves four of their eight products independent of c0. PhiloxRow holds those
+// per-row parts (already xor-ed with the round keys), so a counter of the row
+// costs 18 wide multiplies instead of 20; philox_row_counter() then runs
+// rounds 3..10. The words are bit-identical to philox4x32_10().
+constexpr uint32_t kPhiloxM0 = 0xD2511F53u, kPhiloxM1 = 0xCD9E8D57u;
+constexpr uint32_t kPhiloxW0 = 0x9E3779B9u, kPhiloxW1 = 0xBB67AE85u;
+
+struct PhiloxRow {
+  uint32_t s1;   // c3 ^ k1 (round 1)
+  uint32_t r1k;  // lo(M1 c2) ^ round-2 key 0
+  uint32_t h2k;  // hi(M0 (hi(M1 c2) ^ c1 ^ k0)) ^ round-2 key 1
+  uint32_t l2;   // lo(M0 (hi(M1 c2) ^ c1 ^ k0))
+};
+
+__device__ __forceinline__ PhiloxRow philox_row(uint32_t c1, uint32_t c2, uint32_t c3,
+                                                uint32_t k0, uint32_t k1) {
+  const uint64_t pb = (uint64_t)kPhiloxM1 * c2;
+  const uint32_t x0 = (uint32_t)(pb >> 32) ^ c1 ^ k0;  // word 0 after round 1
+  const uint32_t x1 = (uint32_t)pb;                    // word 1 after round 1
+  const uint64_t p0 = (uint64_t)kPhiloxM0 * x0;        // round 2's first product
+  PhiloxRow r;
+  r.s1 = c3 ^ k1;
+  r.r1k = x1 ^ (k0 + kPhiloxW0);
+  r.h2k = (uint32_t)(p0 >> 32) ^ (k1 + kPhiloxW1);
+  r.l2 = (uint32_t)p0;
+  return r;
+}
+
+__device__ __forceinline__ PhiloxOut philox_row_counter(const PhiloxRow& r, uint32_t c0,
+                                                        uint32_t k0, uint32_t k1) {
+  // round 1: words 0, 1 are row constants; words 2, 3 come from M0 * c0
+  const uint64_t p = (uint64_t)kPhiloxM0 * c0;
+  const uint32_t x2 = (uint32_t)(p >> 32) ^ r.s1, x3 = (uint32_t)p;
+  // round 2: M0 * word 0 is a row constant; M1 * word 2 is not
+  const uint64_t q = (uint64_t)kPhiloxM1 * x2;
+  uint32_t y0 = (uint32_t)(q >> 32) ^ r.r1k, y1 = (uint32_t)q;
+  uint32_t y2 = r.h2k ^ x3, y3 = r.l2;
+#pragma unroll
+  for (int rd = 2; rd < 10; ++rd) {
+    const uint32_t key0 = k0 + (uint32_t)rd * kPhiloxW0, key1 = k1 + (uint32_t)rd * kPhiloxW1;
+    const uint64_t a = (uint64_t)kPhiloxM0 * y0, b = (uint64_t)kPhiloxM1 * y2;
+    const uint32_t n0 = (uint32_t)(b >> 32) ^ y1 ^ key0, n2 = (uint32_t)(a >> 32) ^ y3 ^ key1;
+    y0 = n0; y1 = (uint32_t)b; y2 = n2; y3 = (uint32_t)a;
+  }
+  PhiloxOut o;
+  o.w[0] = y0; o.w[1] = y1; o.w[2] = y2; o.w[3] = y3;
+  return o;
+}
+
+// ---------------------------------------------------------------------------
+// Screening the Gumbel noise of a group of entries without computing it.
+//
+// gumbel_from_word(w) never exceeds kGumbelMax: U <= 1 - 2^-24, so
+// -ln(-ln U) <= -ln(2^-24 (1 + 2^-25)) < 16.6356, and the fp32 evaluation adds
+// far less than the 0.015 of headroom. An entry whose score could only beat a
+// threshold with g > kGumbelMax needs no noise at all.
+constexpr float kGumbelMax = 16.65f;
+
+// For a required noise level G: every word w with gumbel_from_word(w) > G has
+// j(w) + 1/2 < gumbel_screen_limit(G), where j(w) = 2^23 - 1 - (w >> 9) (so
+// that 1 - U = (j + 1/2) 2^-23). Derivation: g > G means
+//   1 - U < 1 - exp(-e^-G) <= e^-G,  i.e.  j + 1/2 < e^-G 2^23,
+// and the limit returned is e^-(G - 0.01) 2^23: the 0.01 covers the fp32
+// evaluation of gumbel_from_word (about 1e-6) and the approximate exp2 here
+// (relative error below 2^-21). Words at or above the limit (in j) are screened
+// out. Checked on the device over all 2^23 noise values by dd_selftest_gumbel_screen.
+constexpr float kScreenSlack = 0.01f;
+__device__ __forceinline__ float gumbel_screen_limit(float G) {
+  return fast_exp2(fmaf(-G, 1.4426950408889634f, 23.f + kScreenSlack * 1.4426950408889634f));
+}
+// j of the largest word among several (the one whose noise could be largest), as
+// an exact float: words w with larger w >> 9 have smaller j.
+__device__ __forceinline__ float gumbel_screen_j(uint32_t wmax) {
+  return __uint_as_float((0x7FFFFFu - (wmax >> 9)) | 0x4B000000u) - 8388608.f;
 }
 
 // Monotone map of floats (no NaN) onto signed integers, for integer max reductions.
@@ -132,11 +206,6 @@ __device__ __forceinline__ float ordered_to_float(int i) {
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-__device__ __forceinline__ float fast_exp2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;

@@ -5,9 +5,11 @@
 // verified row produces: LSE of both, argmax of both, the verifier's max
 // probability, its entropy (the uncertainty u of COVER's seed score),
 // KL(drafter || verifier), and at T > 0 the coupled Gumbel-max samples of both
-// with the same Philox noise (every entry's noise word is drawn, but its exact
-// Gumbel value is computed only where a cheap upper bound says the entry could
-// still be the row's maximum; see fold()).
+// with the same Philox noise. The exact Gumbel value of an entry is computed only
+// where the entry could still be sampled: a 16-byte vector whose logits cannot
+// reach the best score its warp holds even with the largest possible noise draws
+// no noise at all, and one whose generator words all lie below the level it would
+// need is dropped after an integer comparison (see fold()).
 //
 // Work decomposition: the 16-byte vectors of all rows form one index space
 // (rows x vectors per row); it is split into equal contiguous ranges, one per
@@ -120,10 +122,6 @@ __device__ __forceinline__ uint32_t hmax2_bits(uint32_t a, uint32_t b) {
 
 // Fold NV 16-byte vectors of each matrix (vector k starts at vocabulary index v0[k],
 // indices increasing with k). l/m: the unpacked values; lw/mw: the raw words.
-template <typename T, bool SAMPLE, int NV>
-__device__ __forceinline__ void fold(Acc& a, const uint4 (&lw)[NV], const uint4 (&mw)[NV],
-                                     const int (&v0)[NV], int pos, int b, const NoiseKey& key,
-                                     float invT);
 
 template <typename T>
 struct Unpack;
@@ -140,6 +138,11 @@ struct Unpack<__nv_bfloat16> {
     const uint32_t h = hmax2_bits(hmax2_bits(u.x, u.y), hmax2_bits(u.z, u.w));
     return fmaxf(bf16lo(h), bf16hi(h));
   }
+  // entries 2e, 2e + 1 of the vector
+  __device__ static float2 pair(const uint4& u, int e) {
+    const uint32_t w = e == 0 ? u.x : e == 1 ? u.y : e == 2 ? u.z : u.w;
+    return make_float2(bf16lo(w), bf16hi(w));
+  }
 };
 template <>
 struct Unpack<float> {
@@ -152,27 +155,95 @@ struct Unpack<float> {
     return fmaxf(fmaxf(__uint_as_float(u.x), __uint_as_float(u.y)),
                  fmaxf(__uint_as_float(u.z), __uint_as_float(u.w)));
   }
+  __device__ static float2 pair(const uint4& u, int e) {
+    return e == 0 ? make_float2(__uint_as_float(u.x), __uint_as_float(u.y))
+                  : make_float2(__uint_as_float(u.z), __uint_as_float(u.w));
+  }
 };
+
+// ---------------------------------------------------------------------------
+// Exact coupled scores, evaluated by the warp together.
+//
+// A lane whose 16-byte vector passes the noise screen does not evaluate it on its
+// own (that would hold the whole warp for the few lanes that need it); it pushes
+// the vector into its warp's queue in shared memory, and once a few vectors are
+// queued every lane of the warp takes one queued entry at a time: its generator
+// word, its exact fp32 Gumbel value and its two scores. Entries are kept by exact
+// vocabulary index (encoded -1 - v), ties going to the lower index.
+constexpr int kQueueCap = 80;    // vectors per warp
+constexpr int kQueueDrain = 4;   // evaluate once this many vectors are queued
+
+struct NoiseQueue {
+  int v[kQueueCap];             // first vocabulary index of the vector
+  uint4 l[kQueueCap], m[kQueueCap];
+};
+
+__device__ __forceinline__ void keep_best(float& best, int& code, float s, int v) {
+  if (s > best || (s == best && v < -1 - code)) {
+    best = s;
+    code = -1 - v;
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ float vec_entry(const uint4& u, int e) {
+  if constexpr (sizeof(T) == 2) {
+    const uint32_t w = (e >> 1) == 0 ? u.x : (e >> 1) == 1 ? u.y : (e >> 1) == 2 ? u.z : u.w;
+    return (e & 1) ? bf16hi(w) : bf16lo(w);
+  } else {
+    const uint32_t w = e == 0 ? u.x : e == 1 ? u.y : e == 2 ? u.z : u.w;
+    return __uint_as_float(w);
+  }
+}
+
+__device__ __forceinline__ uint32_t pick_word(const PhiloxOut& o, int i) {
+  return i == 0 ? o.w[0] : i == 1 ? o.w[1] : i == 2 ? o.w[2] : o.w[3];
+}
+
+// The exact coupled scores of entry v (logits l, m) into a lane's state.
+__device__ __forceinline__ void exact_entry(Acc& a, int v, float l, float m, const PhiloxRow& pr,
+                                            const NoiseKey& key, float invT) {
+  const PhiloxOut o = philox_row_counter(pr, (uint32_t)(v >> 2), key.k0, key.k1);
+  const float g = gumbel_from_word(pick_word(o, v & 3));
+  keep_best(a.bt, a.vbt, fmaf(l, invT, g), v);
+  keep_best(a.bd, a.vbd, fmaf(m, invT, g), v);
+}
+
+// Every queued entry, spread over the lanes in `act`; empties the queue.
+template <typename T>
+__device__ __noinline__ void drain_queue(Acc& a, NoiseQueue* q, int& qn, unsigned act,
+                                         const PhiloxRow& pr, NoiseKey key, float invT) {
+  constexpr int VEC = Unpack<T>::N;
+  __syncwarp(act);  // the pushes are visible
+  const int lane = threadIdx.x & 31;
+  const int nact = __popc(act), rank = __popc(act & ((1u << lane) - 1u));
+  for (int i = rank; i < qn * VEC; i += nact) {
+    const int s = i / VEC, e = i % VEC;
+    exact_entry(a, q->v[s] + e, vec_entry<T>(q->l[s], e), vec_entry<T>(q->m[s], e), pr, key,
+                invT);
+  }
+  __syncwarp(act);  // every lane is done reading before the queue is reused
+  qn = 0;
+}
 
 template <typename T, bool SAMPLE, int NV>
 __device__ __forceinline__ void fold(Acc& a, const uint4 (&lw)[NV], const uint4 (&mw)[NV],
-                                     const int (&v0)[NV], int pos, int b, const NoiseKey& key,
-                                     float invT) {
+                                     const int (&v0)[NV], const PhiloxRow& pr,
+                                     const NoiseKey& key, float invT, NoiseQueue* q, int& qn) {
   constexpr int VEC = Unpack<T>::N, NP = VEC / 2;
-  float2 L[NV][NP], M[NV][NP];
+  float xm[NV], ym[NV];  // per-vector maxima of l and m
 #pragma unroll
   for (int k = 0; k < NV; ++k) {
-    Unpack<T>::run(lw[k], L[k]);
-    Unpack<T>::run(mw[k], M[k]);
+    xm[k] = Unpack<T>::vmax(lw[k]);
+    ym[k] = Unpack<T>::vmax(mw[k]);
   }
   // --- exact maxima and the first vector holding them (selects, no branch)
-  float cm = Unpack<T>::vmax(lw[0]), dm = Unpack<T>::vmax(mw[0]);
+  float cm = xm[0], dm = ym[0];
   int cv = v0[0], dv = v0[0];
 #pragma unroll
   for (int k = 1; k < NV; ++k) {
-    const float x = Unpack<T>::vmax(lw[k]), y = Unpack<T>::vmax(mw[k]);
-    if (x > cm) { cm = x; cv = v0[k]; }
-    if (y > dm) { dm = y; dv = v0[k]; }
+    if (xm[k] > cm) { cm = xm[k]; cv = v0[k]; }
+    if (ym[k] > dm) { dm = ym[k]; dv = v0[k]; }
   }
   if (cm > a.mt) { a.mt = cm; a.vt = cv; }
   if (dm > a.md) { a.md = dm; a.vd = dv; }
@@ -207,55 +278,66 @@ __device__ __forceinline__ void fold(Acc& a, const uint4 (&lw)[NV], const uint4 
   for (int k = 0; k < NV; ++k)
 #pragma unroll
     for (int e = 0; e < NP; ++e) {
-      const float2 y = __ffma2_rn(L[k][e], l2e, nmt);
+      const float2 lp = Unpack<T>::pair(lw[k], e), mp = Unpack<T>::pair(mw[k], e);
+      const float2 y = __ffma2_rn(lp, l2e, nmt);
       const float2 et = ex2x2(y);
       a.s1t = __fadd2_rn(a.s1t, et);
       a.s2t = __ffma2_rn(et, y, a.s2t);
-      const float2 z = __ffma2_rn(M[k][e], l2e, nmd);
+      const float2 z = __ffma2_rn(mp, l2e, nmd);
       const float2 ed = ex2x2(z);
       a.s1d = __fadd2_rn(a.s1d, ed);
-      a.skd = __ffma2_rn(ed, __ffma2_rn(L[k][e], neg1, M[k][e]), a.skd);
+      a.skd = __ffma2_rn(ed, __ffma2_rn(lp, neg1, mp), a.skd);
     }
-  // --- coupled Gumbel-max samples (same noise for both); best score + its vector.
-  // Screening: a group of four entries needs its exact noise only if an upper
-  // bound of its scores beats the best exact score any lane of the warp has seen
-  // in this row (all lanes work on one row); otherwise none of its scores can be
-  // the row's maximum, nor tie with it. The bound costs one lg2; candidates get
-  // exactly the fp32 noise and scores they always got.
+  // --- coupled Gumbel-max samples (same noise for both).
+  // Screening, per 16-byte vector: thr_t / thr_d are the best exact scores any lane
+  // of the warp holds for this row (all lanes work on one row, and every vector of
+  // this fold lies above every entry evaluated so far, so such a score wins a tie
+  // against any entry here). An entry with noise g scores at most x_max / T + g; it
+  // can only matter if g exceeds G = min over the two matrices of (thr - x_max / T),
+  // minus a rounding slack. If G >= kGumbelMax no noise value can do that and the
+  // vector's generator words are not even drawn; otherwise the words are drawn and
+  // compared, as integers, with the limit that g > G implies (gumbel_screen_limit).
+  // A vector that passes goes to the warp's queue (drain_queue): its entries get
+  // exactly the fp32 noise and scores the unscreened pass would compute.
   if constexpr (SAMPLE) {
     const unsigned act = __activemask();
     const float tht = ordered_to_float(__reduce_max_sync(act, float_to_ordered(a.bt)));
     const float thd = ordered_to_float(__reduce_max_sync(act, float_to_ordered(a.bd)));
-    const float2 it2 = make_float2(invT, invT);
+    // slack for the fp32 rounding of thr - x/T (about 1e-7 relative)
+    const float slt = fmaf(fabsf(tht), 1e-5f, 1e-5f), sld = fmaf(fabsf(thd), 1e-5f, 1e-5f);
+    const float is = invT * 1e-5f;
+    const int lane = threadIdx.x & 31;
+    bool cand[NV];
 #pragma unroll
     for (int k = 0; k < NV; ++k) {
-      float bt = -INFINITY, bd = -INFINITY;
+      const float gt = fmaf(-xm[k], invT, tht) - fmaf(fabsf(xm[k]), is, slt);
+      const float gd = fmaf(-ym[k], invT, thd) - fmaf(fabsf(ym[k]), is, sld);
+      const float G = fminf(gt, gd);
+      cand[k] = false;
+      if (G < kGumbelMax) {
+        uint32_t wm = 0u;
 #pragma unroll
-      for (int q = 0; q < VEC / 4; ++q) {
-        const PhiloxOut o = philox4x32_10((uint32_t)(v0[k] >> 2) + q, (uint32_t)pos,
-                                          (uint32_t)b, key.step, key.k0, key.k1);
-        const float2 u01 = make_float2(gumbel_bound_from_word(o.w[0]), gumbel_bound_from_word(o.w[1]));
-        const float2 u23 = make_float2(gumbel_bound_from_word(o.w[2]), gumbel_bound_from_word(o.w[3]));
-        const float2 s0 = __ffma2_rn(L[k][2 * q], it2, u01);
-        const float2 s1 = __ffma2_rn(L[k][2 * q + 1], it2, u23);
-        const float2 d0 = __ffma2_rn(M[k][2 * q], it2, u01);
-        const float2 d1 = __ffma2_rn(M[k][2 * q + 1], it2, u23);
-        const float ubt = fmaxf(fmaxf(s0.x, s0.y), fmaxf(s1.x, s1.y));
-        const float ubd = fmaxf(fmaxf(d0.x, d0.y), fmaxf(d1.x, d1.y));
-        if (ubt > tht || ubd > thd) {
-          const float2 g01 = make_float2(gumbel_from_word(o.w[0]), gumbel_from_word(o.w[1]));
-          const float2 g23 = make_float2(gumbel_from_word(o.w[2]), gumbel_from_word(o.w[3]));
-          const float2 e0 = __ffma2_rn(L[k][2 * q], it2, g01);
-          const float2 e1 = __ffma2_rn(L[k][2 * q + 1], it2, g23);
-          const float2 f0 = __ffma2_rn(M[k][2 * q], it2, g01);
-          const float2 f1 = __ffma2_rn(M[k][2 * q + 1], it2, g23);
-          bt = fmaxf(bt, fmaxf(fmaxf(e0.x, e0.y), fmaxf(e1.x, e1.y)));
-          bd = fmaxf(bd, fmaxf(fmaxf(f0.x, f0.y), fmaxf(f1.x, f1.y)));
+        for (int qq = 0; qq < VEC / 4; ++qq) {
+          const PhiloxOut o = philox_row_counter(pr, (uint32_t)(v0[k] >> 2) + qq, key.k0, key.k1);
+          wm = max(wm, max(max(o.w[0], o.w[1]), max(o.w[2], o.w[3])));
         }
+        cand[k] = gumbel_screen_j(wm) + 0.5f < gumbel_screen_limit(G);
       }
-      if (bt > a.bt) { a.bt = bt; a.vbt = v0[k]; }
-      if (bd > a.bd) { a.bd = bd; a.vbd = v0[k]; }
     }
+#pragma unroll
+    for (int k = 0; k < NV; ++k) {
+      const unsigned bal = __ballot_sync(act, cand[k]);
+      if (bal) {
+        if (cand[k]) {
+          const int slot = qn + __popc(bal & ((1u << lane) - 1u));
+          q->v[slot] = v0[k];
+          q->l[slot] = lw[k];
+          q->m[slot] = mw[k];
+        }
+        qn += __popc(bal);
+      }
+    }
+    if (qn >= kQueueDrain) drain_queue<T>(a, q, qn, act, pr, key, invT);
   }
 }
 
@@ -349,11 +431,14 @@ __device__ Partial resolve(const Acc& a, const T* lrow, const T* mrow, int pos, 
       float x[VEC], l[VEC], g[VEC];
       Vec<T>::unpack(*reinterpret_cast<const uint4*>(row + vb), x);
       Vec<T>::unpack(*reinterpret_cast<const uint4*>(lrow + vb), l);
+      #pragma unroll
       for (int q = 0; q < VEC / 4; ++q) {
         const PhiloxOut o = philox4x32_10((uint32_t)(vb >> 2) + q, (uint32_t)pos, (uint32_t)b,
                                           key.step, key.k0, key.k1);
+        #pragma unroll
         for (int w = 0; w < 4; ++w) g[4 * q + w] = gumbel_from_word(o.w[w]);
       }
+      #pragma unroll
       for (int e = VEC - 1; e >= 0; --e)
         if (fmaf(x[e], invT, g[e]) == best) {
           idx = vb + e;
@@ -492,6 +577,13 @@ verify_stream_kernel(const VerifyArgs a) {
 
   Acc acc;
   init(acc);
+  // sampling: this warp's queue of vectors awaiting exact noise (see drain_queue)
+  NoiseQueue* q = nullptr;
+  if constexpr (SAMPLE) {
+    __shared__ NoiseQueue queues[kVThreads / 32];
+    q = &queues[cw];
+  }
+  int qn = 0;
   auto flush = [&](int64_t row, Partial p) {
 #pragma unroll
     for (int mask = 16; mask > 0; mask >>= 1) {
@@ -545,14 +637,23 @@ verify_stream_kernel(const VerifyArgs a) {
         }
       }
     };
+    // per-row parts of the noise generator (only used when sampling)
+    const PhiloxRow pr = philox_row((uint32_t)pos, (uint32_t)b, a.key.step, a.key.k0, a.key.k1);
+    // both vectors of a half-step in one fold where both exist (one warp-wide
+    // screening threshold per pair), else the one that does
     auto fold2 = [&](int bs, const uint4 (&l)[2], const uint4 (&m)[2]) {
+      if (SAMPLE && bs + kVThreads < vlim) {
+        const int vv[2] = {bs * VEC, (bs + kVThreads) * VEC};
+        fold<T, SAMPLE, 2>(acc, l, m, vv, pr, a.key, a.invT, q, qn);
+        return;
+      }
 #pragma unroll
       for (int k = 0; k < 2; ++k) {
         const int idx = bs + k * kVThreads;
         if (idx < vlim) {
-          uint4 l1[1] = {l[k]}, m1[1] = {m[k]};
-          int vv[1] = {idx * VEC};
-          fold<T, SAMPLE, 1>(acc, l1, m1, vv, pos, b, a.key, a.invT);
+          const uint4 l1[1] = {l[k]}, m1[1] = {m[k]};
+          const int vv[1] = {idx * VEC};
+          fold<T, SAMPLE, 1>(acc, l1, m1, vv, pr, a.key, a.invT, q, qn);
         }
       }
     };
@@ -560,8 +661,22 @@ verify_stream_kernel(const VerifyArgs a) {
     uint4 la[2], ma[2], lb[2], mb[2];
     int base = vbeg + ct;
     ld2(base, la, ma);
+    bool primed = !SAMPLE;
     for (; base < vlim; base += 2 * kStep) {
       ld2(base + kStep, lb, mb);
+      if (!primed) {
+        // a first exact score per lane (the four entries of its first vector's first
+        // generator counter), so the screen has a threshold from the start
+        primed = true;
+        const int v = base * VEC;
+        const PhiloxOut o = philox_row_counter(pr, (uint32_t)(v >> 2), a.key.k0, a.key.k1);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float g = gumbel_from_word(o.w[e]);
+          keep_best(acc.bt, acc.vbt, fmaf(vec_entry<T>(la[0], e), a.invT, g), v + e);
+          keep_best(acc.bd, acc.vbd, fmaf(vec_entry<T>(ma[0], e), a.invT, g), v + e);
+        }
+      }
       fold2(base, la, ma);
       ld2(base + 2 * kStep, la, ma);
       fold2(base + kStep, lb, mb);
@@ -579,6 +694,14 @@ verify_stream_kernel(const VerifyArgs a) {
         fold_one<SAMPLE>(acc, Vec<T>::scalar(LT + row * a.ld + e),
                          Vec<T>::scalar(LM + row * a.ld + e), g, e, a.invT);
       }
+    }
+    if constexpr (SAMPLE) {
+      // Lanes leave a row piece's last folds in lane order (a lane's vectors lie above
+      // those of the lanes before it), so lane 0 took part in every push: its count
+      // is the warp's. Evaluate what is still queued.
+      __syncwarp();
+      qn = __shfl_sync(0xffffffffu, qn, 0);
+      if (qn > 0) drain_queue<T>(acc, q, qn, 0xffffffffu, pr, a.key, a.invT);
     }
     flush(row, resolve<T, SAMPLE>(acc, LT + row * a.ld, LM + row * a.ld, pos, b, a.key, a.invT));
     sidx += vend - vbeg;
@@ -636,13 +759,31 @@ __global__ void coupled_gumbel_kernel(NoiseKey key, int R, int V, int64_t ld, in
     const int qd = (int)(t % nquads_per_row);
     const int b = (int)(row / R);
     const int pos = pos_offset + (int)(row % R);
-    const PhiloxOut o = philox4x32_10((uint32_t)qd, (uint32_t)pos, (uint32_t)b, key.step,
-                                      key.k0, key.k1);
+    // the row-split generator of the streaming pass, so its words are what the
+    // noise written here is checked against
+    const PhiloxRow pr = philox_row((uint32_t)pos, (uint32_t)b, key.step, key.k0, key.k1);
+    const PhiloxOut o = philox_row_counter(pr, (uint32_t)qd, key.k0, key.k1);
     float* dst = g + row * ld + 4 * (int64_t)qd;
 #pragma unroll
     for (int w = 0; w < 4; ++w)
       if (4 * qd + w < V) dst[w] = gumbel_from_word(o.w[w]);
   }
+}
+
+// Self-test of the noise screen: the fp32 Gumbel value of every noise level
+// k = w >> 9 (2^23 of them), the screen's exact-float j of a word at that level,
+// and the screen limit for each requested noise level.
+__global__ void selftest_gumbel_kernel(float* g_of_k, float* j_of_k, const float* g_req,
+                                       float* limit, int n) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < (1 << 23); t += stride) {
+    const uint32_t k = (uint32_t)t;
+    const uint32_t w = (k << 9) | (k & 511u);  // low bits play no part; mix them anyway
+    g_of_k[t] = gumbel_from_word(w);
+    j_of_k[t] = gumbel_screen_j(w);
+  }
+  for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < n; t += stride)
+    limit[t] = gumbel_screen_limit(g_req[t]);
 }
 
 // Grid and partition for a call (also sizes the workspace).
@@ -728,6 +869,15 @@ cudaError_t launch_verify_logits(const void* lt, const void* lm, dd_dtype dtype,
                 : launch_verify<float, false>(lt, lm, B, R, V, ld, pos_offset, temperature, key,
                                               out, workspace, stream);
 }
+
+cudaError_t launch_selftest_gumbel(float* g_of_k, float* j_of_k, const float* g_req,
+                                   float* limit, int n, cudaStream_t stream) {
+  selftest_gumbel_kernel<<<device_info().sm_count * 4, 256, 0, stream>>>(g_of_k, j_of_k, g_req,
+                                                                        limit, n);
+  return cudaGetLastError();
+}
+
+float gumbel_max_constant() { return kGumbelMax; }
 
 cudaError_t launch_coupled_gumbel(uint64_t seed, uint64_t step, int B, int R, int V, int64_t ld,
                                   int pos_offset, float* g, cudaStream_t stream) {

@@ -28,6 +28,7 @@ EXPORTED = (
     "dd_verify_logits_workspace_size", "dd_verify_logits_static",
     "dd_coupled_gumbel", "dd_select_seeds", "dd_decide", "dd_status_string",
     "dd_get_device_error", "dd_set_spin_limit", "dd_selftest_bounded_wait",
+    "dd_selftest_gumbel_screen",
 )
 
 
@@ -89,6 +90,8 @@ def lib():
     L.dd_set_spin_limit.restype = ctypes.c_uint32
     L.dd_selftest_bounded_wait.argtypes = [ctypes.c_uint32, P]
     L.dd_selftest_bounded_wait.restype = I
+    L.dd_selftest_gumbel_screen.argtypes = [P, P, P, P, I, ctypes.POINTER(F), P]
+    L.dd_selftest_gumbel_screen.restype = I
     _lib = L
     return L
 
@@ -272,3 +275,18 @@ def dd_set_spin_limit(limit: int) -> int:
 def dd_selftest_bounded_wait(spin_limit: int, stream=None):
     _check("dd_selftest_bounded_wait", lib().dd_selftest_bounded_wait(int(spin_limit),
                                                                       _stream(stream)))
+
+
+def dd_selftest_gumbel_screen(g_req, stream=None):
+    """The library's fp32 noise and screen j of every noise level (2^23 each), the
+    screen limit of each requested level g_req (fp32 device tensor), and the
+    constant above which the noise is skipped outright."""
+    dev = g_req.device
+    g = torch.empty(1 << 23, dtype=torch.float32, device=dev)
+    j = torch.empty(1 << 23, dtype=torch.float32, device=dev)
+    limit = torch.empty_like(g_req)
+    gmax = ctypes.c_float(0.0)
+    _check("dd_selftest_gumbel_screen", lib().dd_selftest_gumbel_screen(
+        _ptr(g), _ptr(j), _ptr(g_req), _ptr(limit), g_req.numel(), ctypes.byref(gmax),
+        _stream(stream)))
+    return g, j, limit, float(gmax.value)

@@ -65,13 +65,20 @@ class VerifyStep:
                             pos_offset=s.pos_offset, temperature=s.temperature, seed=self.seed,
                             step=self.step_index, workspace=self.vws)
 
-    def select_and_decide(self):
+    def select(self):
         s, x = self.spec, self.x
         dd.dd_select_seeds(self.stats.entropy_t, s.pos_offset, self.d_in, self.d_out,
                            x["eligible"], self.next_seeds, self.next_is_seed, self.score)
+
+    def decide(self):
+        s, x = self.spec, self.x
         dd.dd_decide(s.policy, x["tokens"], x["is_seed"], x["eligible"], self.stats,
                      s.pos_offset, self.decision, self.new_tokens, self.accepted,
                      tau_kl=s.tau_kl, tau_conf=s.tau_conf, temperature=s.temperature)
+
+    def select_and_decide(self):
+        self.select()
+        self.decide()
 
     def __call__(self):
         self.attention()
@@ -81,8 +88,8 @@ class VerifyStep:
     def forked(self):
         """The same step with the vocabulary pass on a side stream, concurrent with the
         attention call (they share no data; selection needs both, so the streams join
-        before it). The attention kernels leave SMs idle at small shapes and the
-        vocabulary pass fills them."""
+        before it), and the decisions beside the seed selection. The attention kernels
+        leave SMs idle at small shapes and the vocabulary pass fills them."""
         main = torch.cuda.current_stream()
         if self.side is None:
             self.side = torch.cuda.Stream(device=main.device)
@@ -91,7 +98,13 @@ class VerifyStep:
             self.verify()
         self.attention()
         main.wait_stream(self.side)
-        self.select_and_decide()
+        # seed selection (needs both) and the decisions (need only the statistics)
+        # write disjoint outputs: the decisions run beside the selection
+        self.side.wait_stream(main)
+        with torch.cuda.stream(self.side):
+            self.decide()
+        self.select()
+        main.wait_stream(self.side)
 
     def choose_initial_seeds(self):
         """Pass 0 with an empty seed set, then the stability score picks the seeds the

@@ -1,13 +1,73 @@
-"""Host-side arithmetic of bench.py that needs no GPU."""
+"""Host-side pieces of bench.py and of the ncu traffic records that need no GPU."""
+import json
+
+import numpy as np
+import pytest
+
 import bench
+from speculative_verification_cover_b200 import profiling
+from speculative_verification_cover_b200 import workloads as W
 
 
-def test_projection_composes_phases_per_layer():
-    p = bench.projection("llada8b_B1_L512_H32_d128_V126464", 0.04, 0.06, 0.015)
-    assert p["layers"] == 32
-    assert abs(p["ms_per_step"] - (32 * 0.04 + 0.06 + 0.015)) < 1e-12
-    assert abs(p["steps_per_s"] * p["ms_per_step"] - 1000.0) < 1e-9
-    assert "projection" in p["note"]
-    assert bench.projection("dream7b_B8_L2048_H28kv4_d128_V152064", 1, 0, 0)["layers"] == 28
-    assert bench.projection("sdar8b_tree_B16_L1024_H32kv8_d128_V151936", 1, 0, 0)["layers"] == 36
-    assert bench.projection("tiny_f32_B1_L64_H2_d64_V1000", 1, 1, 1) is None
+def test_derived_figures_follow_the_algorithmic_work():
+    spec = W.LLADA8B_L512
+    t = dict(ms=0.1, a_ms=0.04, v_ms=0.05, s_ms=0.01, clocks={})
+    d = bench.derived(spec, t, world=1)
+    vbytes = 2 * 1 * 384 * 126464 * 2
+    assert d["verify"]["algorithmic_bytes"] == vbytes
+    assert d["verify"]["achieved_gbs"] == pytest.approx(vbytes / 0.05e-3 / 1e9)
+    flop = 4 * 32 * 512 ** 2 * 128 + 2 * 32 * 192 * 512 * 128
+    assert d["attention"]["algorithmic_flop"] == flop
+    assert d["attention"]["achieved_tflops"] == pytest.approx(flop / 0.04e-3 / 1e12)
+    assert d["steps_per_s"] == pytest.approx(10000.0)
+    assert d["positions_per_s"] == pytest.approx(10000.0 * 384)
+    # weak scaling: N ranks each doing a batch
+    assert bench.derived(spec, t, world=4)["steps_per_s"] == pytest.approx(40000.0)
+
+
+CSV = '''==PROF== Connected to process 1
+"ID","Kernel Name","dram__bytes_read.sum","dram__bytes_write.sum","gpu__time_duration.sum"
+"","","Mbyte","Kbyte","usecond"
+"0","void dd::verify_stream_kernel<bf16, false>(VerifyArgs)","200.5","3,450.0","49.7"
+"1","void dd::attn_p1_kernel<128>(...)","12.9","4.0","19.7"
+"2","void dd::verify_stream_kernel<bf16, false>(VerifyArgs)","199.5","3,550.0","49.1"
+'''
+
+
+def test_traffic_record_parses_ncu_raw_csv_and_goes_stale(tmp_path):
+    raw = tmp_path / "raw.csv"
+    raw.write_text(CSV)
+    per, n = profiling.dram_bytes_per_launch(str(raw), "verify_stream_kernel")
+    assert n == 2
+    assert per == pytest.approx((200.5e6 + 3.45e6 + 199.5e6 + 3.55e6) / 2)
+    src = tmp_path / "k.cu"
+    src.write_text("// kernel v1\n")
+    out = tmp_path / "traffic.json"
+    rec = profiling.record(str(raw), "verify_stream_kernel", "wl", str(src), "ncu ...",
+                           out=str(out))
+    assert rec["launches"] == 2
+    db = json.loads(out.read_text())
+    assert "verify_stream_kernel@wl" in db
+    # lookup resolves the source relative to the repository root: point it at ours
+    db["verify_stream_kernel@wl"]["source"] = str(src)
+    out.write_text(json.dumps(db))
+    assert profiling.lookup("verify_stream_kernel", "wl", path=str(out)) == pytest.approx(per)
+    assert profiling.lookup("verify_stream_kernel", "other", path=str(out)) is None
+    src.write_text("// kernel v2\n")  # the kernel changed since the capture
+    assert profiling.lookup("verify_stream_kernel", "wl", path=str(out)) is None
+    with pytest.raises(ValueError):
+        profiling.dram_bytes_per_launch(str(raw), "no_such_kernel")
+
+
+def test_oracle_near_tie_counts_on_a_small_sample():
+    spec = W.TINY_F32.replace(temperature=1.0, policy="coupled")
+    x = W.make_inputs(spec, "cpu")
+    near = bench.oracle_near_ties(x, spec, nrows=16)
+    assert near["rows"] == 16
+    assert 0 <= near["near_rows"] <= near["rows"]
+    assert 0 <= near["near_decisions"] <= near["decisions"] <= near["rows"]
+    # the full-step counter of the CPU-baseline leg
+    counts = {}
+    bench.oracle_step(x, spec, 0, near=counts)
+    assert counts["rows"] == spec.R and "seed_boundary_near" in counts
+    assert np.isscalar(counts["near_decisions"])
