@@ -98,3 +98,38 @@ def sequence(q, k_cur, v_cur, k_prev, v_prev, is_seed, is_masked, is_new, scale=
     out, lse, A = dualview_attention(q, k_cur, v_cur, k_prev, v_prev, is_seed, scale)
     masked = np.asarray(is_masked).astype(bool)
     return out, lse, d_in(A[:, masked, :], Hq), d_out(A, is_new, Hq)
+
+
+def layer_stack(layers, is_seed, is_masked, is_new, q_begin=0, scale=None):
+    """A verification pass over several attention layers with a prefix cache.
+
+    [COVER] Results: COVER composes with Fast-dLLM-style prefix caching. Our
+    reading: the K/V rows of the prefix (positions < q_begin, the prompt) come
+    from a cache that was filled once -- they are the given k/v rows, not
+    recomputed -- and the queries of the prefix are not computed at all: only
+    rows >= q_begin produce out and lse. Every layer applies the dual view of
+    [COVER] section 1 with the same seed set. The seed score's statistics of
+    section 2 are averaged over layers: d_in and d_out are the means of the
+    per-layer values (each averaged over heads as in `sequence`); d_out of a
+    prefix row is 0 (its query row is never computed). Seeds and masked
+    positions lie at or after q_begin.
+
+    layers: list of dicts with q [L,Hq,d], k_cur, v_cur, k_prev, v_prev [L,Hkv,d].
+    Returns outs (per layer [L - q_begin, Hq, d]), lses (per layer
+    [Hq, L - q_begin]), d_in [L], d_out [L]."""
+    outs, lses, dins, douts = [], [], [], []
+    masked = np.asarray(is_masked).astype(bool)
+    L = np.asarray(is_masked).shape[0]
+    rows = np.arange(q_begin, L)
+    for x in layers:
+        Hq = np.asarray(x["q"]).shape[1]
+        out, lse, A = dualview_attention(x["q"], x["k_cur"], x["v_cur"], x["k_prev"],
+                                         x["v_prev"], is_seed, scale=scale, rows=rows)
+        # A is [Hq, L - q_begin, L]: masked rows are all >= q_begin
+        dins.append(d_in(A[:, masked[rows], :], Hq))
+        dout = np.zeros(L)
+        dout[rows] = d_out(A, is_new, Hq)
+        douts.append(dout)
+        outs.append(out)
+        lses.append(lse)
+    return outs, lses, np.mean(dins, axis=0), np.mean(douts, axis=0)

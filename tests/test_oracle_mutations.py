@@ -193,3 +193,32 @@ def test_boundary_margin_always_zero_is_caught(monkeypatch):
     monkeypatch.setattr(sd, "boundary_margin", lambda score, k: 0.0)
     assert _fails(TM.test_boundary_margin_special_cases)
     assert _fails(TM.test_boundary_margin_matches_brute_force, 3)
+
+
+# --------------------------------------------------------------------- multi-layer stack
+from tests import test_oracle_layers as TL  # noqa: E402
+
+
+def test_layer_sum_instead_of_mean_is_caught(monkeypatch):
+    orig = att.layer_stack
+
+    def bad(layers, is_seed, is_masked, is_new, q_begin=0, scale=None):
+        outs, lses, din, dout = orig(layers, is_seed, is_masked, is_new, q_begin, scale)
+        return outs, lses, din * len(layers), dout * len(layers)  # bug: summed over layers
+
+    monkeypatch.setattr(att, "layer_stack", bad)
+    assert _fails(TL.test_identical_layers_average_to_one_layer)
+    assert _fails(TL.test_mass_conservation_and_bounds, 2)
+
+
+def test_prefix_rows_computed_anyway_is_caught(monkeypatch):
+    orig = att.layer_stack
+
+    def bad(layers, is_seed, is_masked, is_new, q_begin=0, scale=None):
+        # bug: the prefix's query rows are computed and counted in d_out
+        outs, lses, din, _ = orig(layers, is_seed, is_masked, is_new, 0, scale)
+        _, _, _, dout = orig(layers, is_seed, is_masked, is_new, 0, scale)
+        return [o[q_begin:] for o in outs], [x[:, q_begin:] for x in lses], din, dout
+
+    monkeypatch.setattr(att, "layer_stack", bad)
+    assert _fails(TL.test_prefix_rows_change_nothing_after_them)
