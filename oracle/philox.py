@@ -84,3 +84,18 @@ def gumbel(seed: int, step: int, b: int, pos, v):
     """Standard Gumbel noise g = -ln(-ln U) in fp64 for (b, pos, v)."""
     u = uniform_from_word(noise_words(seed, step, b, pos, v))
     return -np.log(-np.log(u))
+
+
+# Counter word 0 of the decision draws: above every vocabulary counter (v >> 2 < 2^30
+# for any int32 vocabulary index), so a decision draw never reuses sampling noise.
+DECISION_COUNTER = 0x80000000
+
+
+def decision_uniform(seed: int, step: int, b: int, pos: int) -> float:
+    """U of the stochastic decisions at (b, pos): word 0 of Philox4x32-10 at counter
+    (2^31, pos, b, step), mapped like the sampling noise, U = (2 (w >> 9) + 1) 2^-24."""
+    key = (seed & 0xFFFFFFFF, (seed >> 32) & 0xFFFFFFFF)
+    ctr = tuple(np.array([c], dtype=np.uint64) for c in
+                (DECISION_COUNTER, pos, b, step & 0xFFFFFFFF))
+    w = philox4x32_10(ctr, key)[0][0]
+    return float(uniform_from_word(w))

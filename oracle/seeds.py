@@ -10,9 +10,11 @@ remaining masked positions and d_out the drift sensitivity (attention to newly
 written positions).
 
 Our reading where the page is silent: eligible positions are the unmasked
-generated positions (never prompt positions); the set size is a fixed k (the
-page's adaptive size rule is not given); the k highest scores win, ties going
-to the lower position; fewer than k eligible positions leave the tail -1.
+generated positions (never prompt positions); the k highest scores win, ties
+going to the lower position; fewer than k candidates leave the tail -1. The
+page calls the set "small and adaptive" without a rule; our reading of the
+adaptive size: only positions whose score reaches min_score compete, so the
+set holds min(k, #{score >= min_score}) seeds (min_score = -inf: a fixed k).
 """
 from __future__ import annotations
 
@@ -26,10 +28,12 @@ def stability_score(u, d_in, d_out, eligible):
     return np.where(np.asarray(eligible).astype(bool), s, -np.inf)
 
 
-def select(score, k):
-    """Top-k positions by (score descending, position ascending).
-    Returns seeds [k] (rank order, -1 padded) and is_seed [L] uint8."""
+def select(score, k, min_score=-np.inf):
+    """Top-k positions by (score descending, position ascending) among those whose
+    score reaches min_score. Returns seeds [k] (rank order, -1 padded) and is_seed [L]
+    uint8."""
     score = np.asarray(score, dtype=np.float64)
+    score = np.where(score >= min_score, score, -np.inf)
     L = score.shape[0]
     order = np.lexsort((np.arange(L), -score))  # primary key: -score; ties: position
     chosen = [int(i) for i in order[:k] if np.isfinite(score[i])]
@@ -40,9 +44,19 @@ def select(score, k):
     return seeds, is_seed
 
 
-def boundary_margin(score, k):
-    """Gap between the k-th and (k+1)-th finite scores (inf if there is no contest)."""
-    s = np.sort(np.asarray(score, dtype=np.float64)[np.isfinite(score)])[::-1]
+def boundary_margin(score, k, min_score=-np.inf):
+    """Gap between the k-th and (k+1)-th finite scores (inf if there is no contest);
+    with a min_score, also the distance of any finite score to it."""
+    if k == 0:
+        return np.inf
+    score = np.asarray(score, dtype=np.float64)
+    fin = score[np.isfinite(score)]
+    to_min = np.abs(fin - min_score).min() if np.isfinite(min_score) and len(fin) else np.inf
+    s = np.sort(np.where(fin >= min_score, fin, -np.inf))[::-1]
+    s = s[np.isfinite(s)]
+    if len(s) <= k:
+        return to_min
+    return min(s[k - 1] - s[k], to_min)
     if len(s) <= k or k == 0:
         return np.inf
     return s[k - 1] - s[k]

@@ -153,3 +153,15 @@ def test_binding_refuses_cpu_tensors(lib):
     x = torch.zeros(1, 4, 8)
     with pytest.raises(ValueError):
         dd.dd_verify_logits(x, x, dd.RowStats())
+
+
+def test_attention_ex_validation(lib):
+    def ex(q_begin=0, weight=1.0, L=8):
+        return lib.dd_dualview_attention_ex(FAKE, FAKE, FAKE, None, None, None, None, None, 1, L,
+                                            2, 2, 64, 0.0, 1, q_begin, 0, weight, FAKE, FAKE,
+                                            None, None, None, 0, None)
+    assert ex(q_begin=-1) == dd.DD_ERR_INVALID_ARG
+    assert ex(q_begin=8) == dd.DD_ERR_INVALID_ARG          # q_begin must be < L
+    assert ex(weight=float("nan")) == dd.DD_ERR_INVALID_ARG
+    assert ex(weight=float("inf")) == dd.DD_ERR_INVALID_ARG
+    assert ex(L=0) == dd.DD_ERR_INVALID_ARG

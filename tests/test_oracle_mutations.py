@@ -222,3 +222,48 @@ def test_prefix_rows_computed_anyway_is_caught(monkeypatch):
 
     monkeypatch.setattr(att, "layer_stack", bad)
     assert _fails(TL.test_prefix_rows_change_nothing_after_them)
+
+
+# --------------------------------------------------------------------- adaptive seeds, KL draws, commit
+from oracle import decide as dc  # noqa: E402
+from tests import test_oracle_decide_ext as TX  # noqa: E402
+
+
+def test_inverted_kl_probability_is_caught(monkeypatch):
+    orig = dc.decide
+
+    def bad(policy, *a, **kw):  # bug: remask iff U * tau >= KL (probability 1 - KL / tau)
+        d, nt, acc, near = orig(policy, *a, **kw)
+        if policy == "kl_stochastic":
+            flip = (d == dc.KEEP) | (d == dc.REMASK)
+            d = np.where(flip, np.where(d == dc.KEEP, dc.REMASK, dc.KEEP), d).astype(d.dtype)
+        return d, nt, acc, near
+
+    monkeypatch.setattr(dc, "decide", bad)
+    assert _fails(TX.test_kl_stochastic_frequency_is_kl_over_tau, 0.1)
+    assert _fails(TX.test_kl_stochastic_certain_above_threshold_never_at_zero)
+
+
+def test_min_score_strict_is_caught(monkeypatch):
+    orig = sd.select
+    monkeypatch.setattr(sd, "select", lambda score, k, min_score=-np.inf: orig(
+        score, k, np.nextafter(min_score, np.inf)))  # bug: > instead of >=
+    assert _fails(TX.test_adaptive_seed_set_size_and_reduction)
+
+
+def test_commit_tie_to_higher_position_is_caught(monkeypatch):
+    orig = dc.decide
+
+    def bad(*a, **kw):
+        d, nt, acc, near = orig(*a, **kw)
+        tok = np.asarray(a[1])
+        if kw.get("min_commit") and (d == dc.COMMIT).sum() == 1:
+            i = int(np.nonzero(d == dc.COMMIT)[0][0])
+            p = np.asarray(a[4]["p_sample_t"])
+            same = [j for j in range(len(p)) if j > i and tok[j] == -1 and p[j] == p[i]]
+            if same:  # bug: the tie goes to the higher position
+                d[i], d[same[0]] = 0, dc.COMMIT
+        return d, nt, acc, near
+
+    monkeypatch.setattr(dc, "decide", bad)
+    assert _fails(TX.test_commit_progress_rule_and_its_tie)
