@@ -21,6 +21,10 @@ Rank 0 prints one JSON line:
   cpu_baseline  the fp64 CPU oracle on a bounded sample (rank 0, N = 1 only),
             with the oracle's near-tie counts (positions within 1e-4 of a tie or
             a threshold) on that sample
+  multilayer the workload's whole verification pass measured: every attention
+            layer of the model it is shaped like, with and without a prefix cache
+  decode_loop  a synthetic multi-step decode at the workload's shape (N = 1):
+            COVER against confidence remasking, flip-flops and effective revisions
   workloads the other four workloads (N = 1 only; --no-workloads skips them),
             each a few steps: throughput, both rooflines, clocks, near-tie counts
 Under torchrun (N > 1) each rank runs its own batch (weak scaling, no
@@ -61,6 +65,10 @@ def parse():
     p.add_argument("--impl", choices=("ours", "reference"), default="ours")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    p.add_argument("--no-multilayer", action="store_true",
+                   help="skip the measured multi-layer step of the workload")
+    p.add_argument("--no-decode-loop", action="store_true",
+                   help="skip the synthetic multi-step decode (N = 1 only)")
     p.add_argument("--no-workloads", action="store_true",
                    help="skip the per-workload block (the other four workloads, N = 1 only)")
     return p.parse_args()
@@ -369,13 +377,15 @@ def run_e2e(step, x, K, world):
             "d2h_bytes_per_step": d2h}
 
 
-def measure(spec, dev, K, warmup, world, rank, flush):
+def measure(spec, dev, K, warmup, world, rank, flush, x=None, extra_layers=(),
+            prefix_cache=False):
     """Inputs, the step graph, W warm-up and K timed steps of one workload. Returns the
     inputs, the step and the timings (max over ranks)."""
     from speculative_verification_cover_b200 import dd
     from speculative_verification_cover_b200.step import VerifyStep
-    x = W.make_inputs(spec, dev, seed=shard_seed(spec, rank))
-    step = VerifyStep(spec, x)
+    if x is None:
+        x = W.make_inputs(spec, dev, seed=shard_seed(spec, rank))
+    step = VerifyStep(spec, x, extra_layers=extra_layers, prefix_cache=prefix_cache)
     step.choose_initial_seeds()
     step.capture()
     for _ in range(max(warmup, 3)):
@@ -438,6 +448,83 @@ def derived(spec, t, world):
                       "peak_source": f"MEASURED_PEAKS.json bf16_tflops ({peak_src})"},
         "clocks": t["clocks"],
     }
+
+
+# Attention layers of the models the workloads are shaped like: model facts (the
+# pages do not give them), used only to size the measured multi-layer step.
+MODEL_LAYERS = {"llada8b": 32, "dream7b": 28, "sdar8b": 36}
+
+
+def run_multilayer(spec, dev, flush, K, world, rank):
+    """The whole verification pass of a model-shaped step, measured: every attention
+    layer (distinct synthetic operands per layer, d_in / d_out averaged over layers),
+    then the vocabulary pass, seed selection and decisions, as one CUDA graph; with
+    the prompt's K/V rows as a prefix cache (query rows after the prompt only) and
+    without it."""
+    from speculative_verification_cover_b200 import dd
+    n = MODEL_LAYERS.get(spec.name.split("_")[0])
+    if n is None:
+        return None
+    x = W.make_inputs(spec, dev, seed=shard_seed(spec, rank))
+    extra = W.layer_operands(spec, dev, seed=4242 + rank, n_layers=n - 1)
+    _, _, bf16, _ = peaks()
+    res = {"layers": n, "layers_source": "model fact (not on the pages)",
+           "operands": "distinct seeded synthetic q/k/v per layer"}
+    for prefix in (True, False):
+        _, step, t = measure(spec, dev, K, 3, world, rank, flush, x=x, extra_layers=extra,
+                             prefix_cache=prefix)
+        rows = spec.L - (spec.prompt if prefix else 0)
+        masked = spec.masked if not spec.tree else spec.block - 1
+        flop = n * (4 * spec.B * spec.Hq * rows * spec.L * spec.d
+                    + 2 * spec.B * spec.Hq * masked * spec.L * spec.d)
+        res["prefix_cache" if prefix else "no_cache"] = {
+            "q_begin": step.q_begin, "ms_per_step": t["ms"],
+            "steps_per_s": world * 1000.0 / t["ms"],
+            "positions_per_s": world * 1000.0 / t["ms"] * spec.B * spec.R,
+            "attention_ms": t["a_ms"], "verify_ms": t["v_ms"], "select_decide_ms": t["s_ms"],
+            "attention_tflops": flop / (t["a_ms"] * 1e-3) / 1e12,
+            "attention_frac": flop / (t["a_ms"] * 1e-3) / 1e12 / bf16,
+            "attention_algorithmic_flop": flop, "gpu_launches_per_step": step.kernels_per_step,
+            "clocks": t["clocks"]}
+        step.graphs = None
+        del step
+        torch.cuda.empty_cache()
+    assert dd.dd_get_device_error() == dd.DD_OK
+    return res
+
+
+def run_decode_loop(spec, dev, max_steps=96):
+    """The synthetic multi-step decode at this workload's shape: COVER (dual view,
+    stability-selected seeds, KEEP / REPLACE / REMASK on seeds) against confidence
+    remasking of every drafted token without the dual view, both with dynamic
+    threshold commits. Reports decode steps, the library's device time per step and
+    the revision diagnostics (flip-flops, effective-revision ratio)."""
+    from speculative_verification_cover_b200 import dd
+    from speculative_verification_cover_b200.decode_loop import (DecodeLoop, LoopConfig,
+                                                                 revision_metrics)
+    if spec.tree:
+        return None
+    res = {"dynamics": "synthetic (workloads.DecodeDynamics: hidden targets, verifier "
+                       "confidence and accuracy grow with the correct context)",
+           "max_steps": max_steps}
+    for name, cfg in (("cover", LoopConfig(policy="cover", use_seeds=True, k=max(spec.k, 1),
+                                           tau_conf=spec.tau_conf)),
+                      ("conf_remask", LoopConfig(policy="conf", use_seeds=False,
+                                                 tau_conf=spec.tau_conf))):
+        dyn = W.DecodeDynamics(spec, dev, seed=99)
+        loop = DecodeLoop(spec, dyn, cfg)
+        trace = loop.run(max_steps)
+        m = revision_metrics(trace)
+        ms = float(np.median(trace.lib_ms))
+        P = spec.prompt
+        m.update(lib_ms_per_step=ms, lib_steps_per_s=1000.0 / ms, completed=loop.done(),
+                 final_accuracy=float((loop.tokens[:, P:].long() == dyn.target[:, P:])
+                                      .float().mean()))
+        res[name] = m
+        del loop, dyn
+        torch.cuda.empty_cache()
+    assert dd.dd_get_device_error() == dd.DD_OK
+    return res
 
 
 def run_workloads_block(args, dev, flush, with_oracle):
@@ -518,6 +605,10 @@ def run_ours(args, world, rank, local):
     step.graphs = None  # release graphs before the process group
     del x, step
     torch.cuda.empty_cache()
+    if not args.no_multilayer:
+        line["multilayer"] = run_multilayer(spec, dev, flush, max(3, min(K, 20)), world, rank)
+    if world == 1 and not args.no_decode_loop:
+        line["decode_loop"] = run_decode_loop(spec, dev)
     if world == 1 and not args.no_workloads:
         line["workloads"] = run_workloads_block(args, dev, flush, with_oracle)
     if rank == 0:

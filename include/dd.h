@@ -63,11 +63,12 @@ typedef enum {
   DD_POLICY_KL = 1,       /* [DD] KL Divergence-based Remasking */
   DD_POLICY_CONF = 2,     /* [DD] Confidence-based Remasking */
   DD_POLICY_COVER = 3,    /* [COVER] section 3, KEEP / REPLACE / REMASK on seeds */
-  DD_POLICY_COUPLED = 4   /* [SPOT] Coupled-Noise Verification */
+  DD_POLICY_COUPLED = 4,  /* [SPOT] Coupled-Noise Verification */
+  DD_POLICY_KL_STOCHASTIC = 5  /* [DD] KL remasking, "or probabilistically high" */
 } dd_policy;
 
 /* Decision codes written by dd_decide. */
-enum { DD_NONE = 0, DD_KEEP = 1, DD_REPLACE = 2, DD_REMASK = 3 };
+enum { DD_NONE = 0, DD_KEEP = 1, DD_REPLACE = 2, DD_REMASK = 3, DD_COMMIT = 4 };
 #define DD_MASK_TOKEN (-1)
 
 /*
@@ -112,6 +113,37 @@ dd_status dd_dualview_attention(
     const uint8_t* is_seed, const uint8_t* is_masked, const uint8_t* is_new,
     int B, int L, int Hq, int Hkv, int d, float softmax_scale, dd_dtype dtype,
     int accumulate_stats,
+    void* out, float* lse, float* d_in, float* d_out,
+    void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * dd_dualview_attention_ex -- dd_dualview_attention for one layer of a
+ * multi-layer verification pass with a prefix cache ([COVER] Results: COVER
+ * composes with Fast-dLLM-style prefix caching; section 2's statistics are
+ * taken over the whole pass).
+ *   q_begin       first query row computed, 0 <= q_begin < L. Rows before it are
+ *                 a cached prefix (the prompt): their K/V rows in k_cur / v_cur
+ *                 (and k_prev / v_prev) were filled once from the cache and are
+ *                 read as keys, but their queries are not computed -- out and lse
+ *                 rows before q_begin are not written (q rows there are not read),
+ *                 and they contribute 0 to d_out. Seeds and masked positions must
+ *                 lie at or after q_begin.
+ *   stats_weight  this layer's d_in / d_out are multiplied by it before they are
+ *                 written (accumulate_stats = 0) or added (accumulate_stats = 1):
+ *                 1 / n_layers on every layer of an n-layer pass, with
+ *                 accumulate_stats = 0 on the first and 1 on the rest, leaves the
+ *                 layer average. Finite.
+ * Every other argument as dd_dualview_attention, which is this call with
+ * q_begin = 0 and stats_weight = 1.
+ * Errors: as dd_dualview_attention; DD_ERR_INVALID_ARG for q_begin outside
+ * [0, L) or a non-finite stats_weight.
+ */
+dd_status dd_dualview_attention_ex(
+    const void* q, const void* k_cur, const void* v_cur,
+    const void* k_prev, const void* v_prev,
+    const uint8_t* is_seed, const uint8_t* is_masked, const uint8_t* is_new,
+    int B, int L, int Hq, int Hkv, int d, float softmax_scale, dd_dtype dtype,
+    int q_begin, int accumulate_stats, float stats_weight,
     void* out, float* lse, float* d_in, float* d_out,
     void* workspace, size_t workspace_bytes, void* stream);
 
@@ -186,6 +218,9 @@ size_t dd_verify_logits_workspace_size(int B, int R, int V, dd_dtype dtype);
  * without the workspace.
  *   - The first call on a device looks up that array's device address (with
  *     that device current); make that first call before any stream capture.
+ *     The address is kept for the life of the process: after cudaDeviceReset (or
+ *     anything else that tears the device's context down) this entry point must
+ *     not be called again on that device.
  *   - Every call shares the one array and leaves its contents behind; nothing in
  *     it needs to start at zero. Calls that overlap on the GPU (e.g. on two
  *     streams, or two threads) race on it: serialise them.
@@ -235,6 +270,10 @@ typedef struct {
   float tau_kl;       /* KL threshold (REMASK if KL > tau_kl); <= 0 disables it for COUPLED */
   float tau_conf;     /* confidence threshold (CONF: REMASK if conf < tau; COVER: REPLACE if p >= tau) */
   float temperature;  /* > 0: pred = sample_t; 0: pred = argmax_t */
+  float tau_commit;   /* > 0: dynamic threshold decoding on masked positions (see dd_decide) */
+  int min_commit;     /* 1: commit at least one masked position per sequence (see dd_decide) */
+  uint64_t seed;      /* key of the stochastic decisions' draws (KL_STOCHASTIC) */
+  uint64_t step;      /* their step counter (low 32 bits used) */
 } dd_decide_params;
 
 /*
@@ -246,6 +285,18 @@ typedef struct {
  *   COVER   seeds:    pred == token -> KEEP; p_t(pred) >= tau_conf -> REPLACE(pred); else REMASK
  *   COUPLED eligible: sample_d == pred -> KEEP(pred); else tau_kl > 0 and
  *                     kl_dt > tau_kl -> REMASK; else REPLACE(pred)
+ *   KL_STOCHASTIC eligible: REMASK if U * tau_kl < kl_dt (fp32), else KEEP: certain
+ *                     when kl_dt > tau_kl, else with probability kl_dt / tau_kl. U is
+ *                     the uniform of Philox4x32-10 word 0 at counter
+ *                     (2^31, position, b, step lo32), key (seed lo32, seed hi32),
+ *                     U = (2*(word >> 9) + 1) * 2^-24 (the mapping of the sampling
+ *                     noise; counter word 2^31 is never a vocabulary counter).
+ * Dynamic threshold decoding ([SPOT] section 3, SPOT-Sets with dynamic threshold
+ * decoding), on still-masked positions (token DD_MASK_TOKEN) with a verified row,
+ * whatever the policy: with tau_commit > 0, p_sample_t >= tau_commit -> DD_COMMIT
+ * with new token pred; with min_commit = 1, a sequence none of whose masked
+ * positions passes commits its single most confident one (lowest position on a
+ * tie), so every step unmasks something. COMMIT does not enter accepted[b].
  * Only positions with a verified row are decided; others get DD_NONE and keep
  * their token. new_tokens: KEEP keeps the token (COUPLED: the agreed sample),
  * REPLACE writes pred, REMASK writes DD_MASK_TOKEN.
@@ -263,6 +314,20 @@ dd_status dd_decide(
     uint8_t* decision, int32_t* new_tokens, uint8_t* accepted, void* stream);
 
 /* Human-readable name of a status. */
+/*
+ * dd_select_seeds_ex -- dd_select_seeds with an adaptive set size ([COVER]
+ * section 2 calls the seed set "small and adaptive"; the page gives no rule).
+ * Only positions whose fp32 score reaches min_score compete, so each sequence
+ * gets min(k, #{score >= min_score}) seeds; -INFINITY gives dd_select_seeds.
+ * count  [B] int32 out (may be NULL): seeds chosen per sequence.
+ * Errors: as dd_select_seeds; DD_ERR_INVALID_ARG for a NaN min_score.
+ */
+dd_status dd_select_seeds_ex(
+    const float* entropy, int R, int pos_offset,
+    const float* d_in, const float* d_out, const uint8_t* eligible,
+    int B, int L, int k, float min_score, int32_t* seeds, uint8_t* is_seed, float* score,
+    int32_t* count, void* stream);
+
 const char* dd_status_string(dd_status s);
 
 /* Synchronises `stream`, then returns and clears the device error word

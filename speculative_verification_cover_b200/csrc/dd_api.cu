@@ -68,14 +68,16 @@ size_t dd_dualview_attention_workspace_size(int B, int L, int Hq, int Hkv, int d
   return attn_workspace_layout(B, L, Hq, Hkv, d).total;
 }
 
-dd_status dd_dualview_attention(const void* q, const void* k_cur, const void* v_cur,
-                                const void* k_prev, const void* v_prev, const uint8_t* is_seed,
-                                const uint8_t* is_masked, const uint8_t* is_new, int B, int L,
-                                int Hq, int Hkv, int d, float softmax_scale, dd_dtype dtype,
-                                int accumulate_stats, void* out, float* lse, float* d_in,
-                                float* d_out, void* workspace, size_t workspace_bytes,
-                                void* stream) {
+dd_status dd_dualview_attention_ex(const void* q, const void* k_cur, const void* v_cur,
+                                   const void* k_prev, const void* v_prev, const uint8_t* is_seed,
+                                   const uint8_t* is_masked, const uint8_t* is_new, int B, int L,
+                                   int Hq, int Hkv, int d, float softmax_scale, dd_dtype dtype,
+                                   int q_begin, int accumulate_stats, float stats_weight,
+                                   void* out, float* lse, float* d_in, float* d_out,
+                                   void* workspace, size_t workspace_bytes, void* stream) {
   if (!q || !k_cur || !v_cur || !out || !lse) return DD_ERR_INVALID_ARG;
+  if (q_begin < 0 || q_begin >= L) return DD_ERR_INVALID_ARG;
+  if (!(stats_weight == stats_weight) || isinf(stats_weight)) return DD_ERR_INVALID_ARG;
   if (is_seed && (!k_prev || !v_prev)) return DD_ERR_INVALID_ARG;
   if (B < 1 || L < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return DD_ERR_INVALID_ARG;
   if (B > 65535 || Hq > 65535) return DD_ERR_UNSUPPORTED;
@@ -96,6 +98,8 @@ dd_status dd_dualview_attention(const void* q, const void* k_cur, const void* v_
   a.scale = softmax_scale > 0.f ? softmax_scale : 1.f / sqrtf((float)d);
   a.dtype = dtype;
   a.accumulate = accumulate_stats ? 1 : 0;
+  a.q_begin = q_begin;
+  a.stats_weight = stats_weight;
   a.out = out; a.lse = lse; a.d_in = d_in; a.d_out = d_out;
   char* w = static_cast<char*>(workspace);
   a.dout_part = reinterpret_cast<float*>(w + ws.dout_off);
@@ -110,6 +114,19 @@ dd_status dd_dualview_attention(const void* q, const void* k_cur, const void* v_
   a.lse2_m = reinterpret_cast<float*>(w + ws.lse2m_off);
   a.Lp = ws.Lp;
   return from_cuda(launch_attention(a, static_cast<cudaStream_t>(stream)));
+}
+
+dd_status dd_dualview_attention(const void* q, const void* k_cur, const void* v_cur,
+                                const void* k_prev, const void* v_prev, const uint8_t* is_seed,
+                                const uint8_t* is_masked, const uint8_t* is_new, int B, int L,
+                                int Hq, int Hkv, int d, float softmax_scale, dd_dtype dtype,
+                                int accumulate_stats, void* out, float* lse, float* d_in,
+                                float* d_out, void* workspace, size_t workspace_bytes,
+                                void* stream) {
+  if (L < 1) return DD_ERR_INVALID_ARG;
+  return dd_dualview_attention_ex(q, k_cur, v_cur, k_prev, v_prev, is_seed, is_masked, is_new, B,
+                                  L, Hq, Hkv, d, softmax_scale, dtype, 0, accumulate_stats, 1.f,
+                                  out, lse, d_in, d_out, workspace, workspace_bytes, stream);
 }
 
 size_t dd_verify_logits_workspace_size(int B, int R, int V, dd_dtype dtype) {
@@ -144,17 +161,27 @@ dd_status dd_coupled_gumbel(uint64_t seed, uint64_t step, int B, int R, int V, i
       launch_coupled_gumbel(seed, step, B, R, V, ld, pos_offset, g, static_cast<cudaStream_t>(stream)));
 }
 
-dd_status dd_select_seeds(const float* entropy, int R, int pos_offset, const float* d_in,
-                          const float* d_out, const uint8_t* eligible, int B, int L, int k,
-                          int32_t* seeds, uint8_t* is_seed, float* score, void* stream) {
+dd_status dd_select_seeds_ex(const float* entropy, int R, int pos_offset, const float* d_in,
+                             const float* d_out, const uint8_t* eligible, int B, int L, int k,
+                             float min_score, int32_t* seeds, uint8_t* is_seed, float* score,
+                             int32_t* count, void* stream) {
   if (!d_in || !d_out || !eligible) return DD_ERR_INVALID_ARG;
+  if (!(min_score == min_score)) return DD_ERR_INVALID_ARG;
   if (B < 1 || L < 1 || k < 0 || R < 0 || pos_offset < 0) return DD_ERR_INVALID_ARG;
   if (R > 0 && !entropy) return DD_ERR_INVALID_ARG;
   if (k > 0 && !seeds) return DD_ERR_INVALID_ARG;
   if (k > kSelectMaxK || L > kSelectMaxL) return DD_ERR_UNSUPPORTED;
   if (B > 2147483647 / 1) return DD_ERR_UNSUPPORTED;
   return from_cuda(launch_select_seeds(entropy, R, pos_offset, d_in, d_out, eligible, B, L, k,
-                                       seeds, is_seed, score, static_cast<cudaStream_t>(stream)));
+                                       min_score, seeds, is_seed, score, count,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+dd_status dd_select_seeds(const float* entropy, int R, int pos_offset, const float* d_in,
+                          const float* d_out, const uint8_t* eligible, int B, int L, int k,
+                          int32_t* seeds, uint8_t* is_seed, float* score, void* stream) {
+  return dd_select_seeds_ex(entropy, R, pos_offset, d_in, d_out, eligible, B, L, k, -INFINITY,
+                            seeds, is_seed, score, nullptr, stream);
 }
 
 dd_status dd_decide(const dd_decide_params* params, const int32_t* tokens,
@@ -165,6 +192,9 @@ dd_status dd_decide(const dd_decide_params* params, const int32_t* tokens,
   if (B < 1 || L < 1 || R < 0 || pos_offset < 0) return DD_ERR_INVALID_ARG;
   const dd_decide_params& p = *params;
   if (!(p.temperature >= 0.f)) return DD_ERR_INVALID_ARG;
+  if (!(p.tau_commit == p.tau_commit) || p.min_commit < 0 || p.min_commit > 1)
+    return DD_ERR_INVALID_ARG;
+  if (p.tau_commit > 0.f && !stats->p_sample_t) return DD_ERR_INVALID_ARG;
   const bool sampled = p.temperature > 0.f;
   if (sampled ? !stats->sample_t : !stats->argmax_t) return DD_ERR_INVALID_ARG;
   switch (p.policy) {
@@ -183,6 +213,9 @@ dd_status dd_decide(const dd_decide_params* params, const int32_t* tokens,
     case DD_POLICY_COUPLED:
       if (!eligible || (sampled ? !stats->sample_d : !stats->argmax_d)) return DD_ERR_INVALID_ARG;
       if (p.tau_kl > 0.f && !stats->kl_dt) return DD_ERR_INVALID_ARG;
+      break;
+    case DD_POLICY_KL_STOCHASTIC:
+      if (!eligible || !stats->kl_dt || !(p.tau_kl > 0.f)) return DD_ERR_INVALID_ARG;
       break;
     default:
       return DD_ERR_INVALID_ARG;

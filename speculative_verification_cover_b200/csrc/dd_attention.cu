@@ -137,6 +137,7 @@ struct HeadReduce {
   const float* part;
   int nslices;
   float* dst;
+  int begin;  // positions before it have no partials: they contribute 0
 };
 __global__ void __launch_bounds__(256) head_reduce_kernel(HeadReduce r0, HeadReduce r1, int B, int L,
                                                           float inv_hq, int accumulate) {
@@ -153,7 +154,8 @@ __global__ void __launch_bounds__(256) head_reduce_kernel(HeadReduce r0, HeadRed
     if (r.part == nullptr) continue;
     const float* p = r.part + b * r.nslices * L + j;
     float acc = 0.f;
-    for (int h = sub; h < r.nslices; h += 8) acc += p[(int64_t)h * L];
+    if (j >= r.begin)
+      for (int h = sub; h < r.nslices; h += 8) acc += p[(int64_t)h * L];
     acc += __shfl_xor_sync(mask, acc, 4);
     acc += __shfl_xor_sync(mask, acc, 2);
     acc += __shfl_xor_sync(mask, acc, 1);
@@ -220,7 +222,7 @@ __global__ void __launch_bounds__(128) simt_pass1_kernel(AttnArgs a) {
   const int b = blockIdx.z, h = blockIdx.y;
   const int G = a.Hq / a.Hkv, g = h / G;
   const int r = threadIdx.x >> 2, qd = threadIdx.x & 3;
-  const int i = blockIdx.x * kRows + r;
+  const int i = a.q_begin + blockIdx.x * kRows + r;
   const bool valid = i < a.L;
   const int L = a.L;
   const T* qp = static_cast<const T*>(a.q);
@@ -406,7 +408,7 @@ __global__ void __launch_bounds__(128) simt_pass2_kernel(AttnArgs a) {
 
 template <typename T, int D>
 cudaError_t launch_simt(const AttnArgs& a, cudaStream_t stream) {
-  dim3 g1((a.L + kRows - 1) / kRows, a.Hq, a.B);
+  dim3 g1((a.L - a.q_begin + kRows - 1) / kRows, a.Hq, a.B);
   simt_pass1_kernel<T, D><<<g1, 128, 0, stream>>>(a);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
@@ -466,18 +468,18 @@ cudaError_t launch_attention(const AttnArgs& a, cudaStream_t stream) {
     if (err != cudaSuccess) return err;
   }
   const int64_t total = (int64_t)a.B * a.L;
-  HeadReduce rin{nullptr, 0, nullptr}, rout{nullptr, 0, nullptr};
+  HeadReduce rin{nullptr, 0, nullptr, 0}, rout{nullptr, 0, nullptr, 0};
   if (a.d_out) {
-    if (a.is_new) rout = HeadReduce{a.dout_part, a.Hq, a.d_out};
+    if (a.is_new) rout = HeadReduce{a.dout_part, a.Hq, a.d_out, a.q_begin};
     else if (!a.accumulate) cudaMemsetAsync(a.d_out, 0, total * sizeof(float), stream);
   }
   if (a.d_in) {
-    if (need_din) rin = HeadReduce{a.din_part, din_slices, a.d_in};
+    if (need_din) rin = HeadReduce{a.din_part, din_slices, a.d_in, 0};
     else if (!a.accumulate) cudaMemsetAsync(a.d_in, 0, total * sizeof(float), stream);
   }
   if (rin.part || rout.part) {
     head_reduce_kernel<<<(unsigned)((total * 8 + 255) / 256), 256, 0, stream>>>(
-        rin, rout, a.B, a.L, 1.f / a.Hq, a.accumulate);
+        rin, rout, a.B, a.L, a.stats_weight / a.Hq, a.accumulate);
   }
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   return cudaSuccess;

@@ -79,6 +79,7 @@ struct P1Params {
   const uint32_t* newbits;  // [B, ceil(L/32)]
   const int32_t* mrank;     // [B, L]
   int L, Hq, Hkv, Lp;
+  int q_begin;  // first query row (rows before it are a cached prefix, not computed)
   float scale_log2;
   __nv_bfloat16* out;
   float* lse;
@@ -106,7 +107,7 @@ attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int L = p.L;
   const int g = h / (p.Hq / p.Hkv);
-  const int q0 = qt * kBM;
+  const int q0 = p.q_begin + qt * kBM;
   const int T = (L + kBN - 1) / kBN;
   volatile int* abort_flag = &bars->abort_flag;
 
@@ -308,10 +309,12 @@ attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         for (int c = 0; c < kBN; ++c)
           if (j * kBN + c >= L) s[c] = -INFINITY;
       }
-      if (seed_row && j == qt) {
+      if (seed_row && j == i / kBN) {
+        // the seed's own column (query tiles need not line up with key tiles)
+        const int sc = i & (kBN - 1);
 #pragma unroll
         for (int c = 0; c < kBN; ++c)
-          if (c == r) s[c] = -INFINITY;
+          if (c == sc) s[c] = -INFINITY;
       }
       // row maximum: eight independent chains of three-input maxima, then a tree
       float pm[8];
@@ -726,6 +729,7 @@ cudaError_t launch_p1(const AttnArgs& a, bool pass2, cudaStream_t stream) {
   p.Hq = a.Hq;
   p.Hkv = a.Hkv;
   p.Lp = a.Lp;
+  p.q_begin = a.q_begin;
   p.scale_log2 = a.scale * kLog2e;
   p.out = static_cast<__nv_bfloat16*>(a.out);
   p.lse = a.lse;
@@ -742,7 +746,7 @@ cudaError_t launch_p1(const AttnArgs& a, bool pass2, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     configured[di.device & 63] = 1;
   }
-  dim3 grid((a.L + kBM - 1) / kBM, a.Hq, a.B);
+  dim3 grid((a.L - a.q_begin + kBM - 1) / kBM, a.Hq, a.B);
   attn_p1_kernel<D><<<grid, kP1Threads, smem, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }

@@ -28,6 +28,8 @@ struct AttnArgs {
   float scale;          // softmax scale (natural units)
   dd_dtype dtype;
   int accumulate;
+  int q_begin;          // first query row computed (rows before it: a cached prefix)
+  float stats_weight;   // this call's d_in / d_out are added with this weight
   void* out;
   float* lse;
   float *d_in, *d_out;
@@ -66,8 +68,8 @@ cudaError_t launch_coupled_gumbel(uint64_t seed, uint64_t step, int B, int R, in
 
 cudaError_t launch_select_seeds(const float* entropy, int R, int pos_offset, const float* d_in,
                                 const float* d_out, const uint8_t* eligible, int B, int L, int k,
-                                int32_t* seeds, uint8_t* is_seed, float* score,
-                                cudaStream_t stream);
+                                float min_score, int32_t* seeds, uint8_t* is_seed, float* score,
+                                int32_t* count, cudaStream_t stream);
 
 cudaError_t launch_decide(const dd_decide_params& p, const int32_t* tokens,
                           const uint8_t* is_seed, const uint8_t* eligible,

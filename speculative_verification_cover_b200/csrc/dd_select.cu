@@ -52,9 +52,9 @@ __device__ __forceinline__ int block_exclusive_sum(int x, int* warp_tmp, int* to
 __global__ void __launch_bounds__(kSelThreads)
 select_seeds_kernel(const float* __restrict__ entropy, int R, int pos_offset,
                     const float* __restrict__ d_in, const float* __restrict__ d_out,
-                    const uint8_t* __restrict__ eligible, int L, int k,
+                    const uint8_t* __restrict__ eligible, int L, int k, float min_score,
                     int32_t* __restrict__ seeds, uint8_t* __restrict__ is_seed,
-                    float* __restrict__ score) {
+                    float* __restrict__ score, int32_t* __restrict__ count) {
   extern __shared__ uint32_t skey[];  // [L] orderable score; 0 = not a candidate
   __shared__ unsigned int hist[256];
   __shared__ int warp_tmp[32];
@@ -76,8 +76,10 @@ select_seeds_kernel(const float* __restrict__ entropy, int R, int pos_offset,
     if (eligible[bi] && r >= 0 && r < R) {
       const float u = entropy[(int64_t)b * R + r];
       s = u * (1.f + d_in[bi]) / (1.f + d_out[bi]);
-      key = orderable(s);
-      ++my_cand;
+      if (s >= min_score) {  // the adaptive set: only scores reaching the floor compete
+        key = orderable(s);
+        ++my_cand;
+      }
     }
     skey[i] = key;
     if (score) score[bi] = s;
@@ -158,9 +160,13 @@ select_seeds_kernel(const float* __restrict__ entropy, int R, int pos_offset,
     seeds[(int64_t)b * k + rank] = (int32_t)(0xFFFFFFFFu - (uint32_t)(key & 0xFFFFFFFFull));
   }
   for (int t = nsel + threadIdx.x; t < k; t += blockDim.x) seeds[(int64_t)b * k + t] = -1;
+  if (count && threadIdx.x == 0) count[b] = nsel;
 }
 
-// One CTA per sequence; accepted[b] = all decided positions KEEP.
+// One CTA per sequence; accepted[b] = all decided positions of the policy's domain
+// KEEP. Dynamic threshold decoding commits masked positions with p(pred) >= tau_commit;
+// with min_commit, a sequence where none does commits its most confident one (a
+// block-wide max of (p, -position) keys).
 __global__ void __launch_bounds__(1024)
 decide_kernel(dd_decide_params p, const int32_t* __restrict__ tokens,
               const uint8_t* __restrict__ is_seed, const uint8_t* __restrict__ eligible,
@@ -168,7 +174,11 @@ decide_kernel(dd_decide_params p, const int32_t* __restrict__ tokens,
               int32_t* __restrict__ new_tokens, uint8_t* __restrict__ accepted) {
   const int b = blockIdx.x;
   const bool sampled = p.temperature > 0.f;
-  int all_keep = 1;
+  const bool commit_on = p.tau_commit > 0.f;
+  __shared__ unsigned long long best_key;  // most confident masked position: (p, -pos)
+  if (threadIdx.x == 0) best_key = 0ull;
+  __syncthreads();
+  int all_keep = 1, committed = 0;
   for (int i = threadIdx.x; i < L; i += blockDim.x) {
     const int64_t bi = (int64_t)b * L + i;
     const int r = i - pos_offset;
@@ -201,18 +211,45 @@ decide_kernel(dd_decide_params p, const int32_t* __restrict__ tokens,
           else dcs = DD_REPLACE;
           break;
         }
+        case DD_POLICY_KL_STOCHASTIC: {
+          // REMASK with probability min(1, KL / tau), decided as U * tau < KL in fp32
+          const PhiloxOut o = philox4x32_10(0x80000000u, (uint32_t)i, (uint32_t)b,
+                                            (uint32_t)p.step, (uint32_t)p.seed,
+                                            (uint32_t)(p.seed >> 32));
+          const float u = uniform_from_word(o.w[0]);
+          dcs = __fmul_rn(u, p.tau_kl) < st.kl_dt[row] ? DD_REMASK : DD_KEEP;
+          break;
+        }
         default:
           break;
       }
       if (dcs == DD_REPLACE || (dcs == DD_KEEP && p.policy == DD_POLICY_COUPLED)) tok = pred;
       else if (dcs == DD_REMASK) tok = DD_MASK_TOKEN;
       if (dcs != DD_KEEP) all_keep = 0;
+    } else if (commit_on && cur == DD_MASK_TOKEN && r >= 0 && r < R) {
+      const int64_t row = (int64_t)b * R + r;
+      const float pp = st.p_sample_t[row];
+      if (pp >= p.tau_commit) {
+        dcs = DD_COMMIT;
+        tok = sampled ? st.sample_t[row] : st.argmax_t[row];
+        committed = 1;
+      } else if (p.min_commit) {
+        atomicMax(&best_key, ((unsigned long long)orderable(pp) << 32) | (0xFFFFFFFFu - (uint32_t)i));
+      }
     }
     decision[bi] = dcs;
     new_tokens[bi] = tok;
   }
   const int acc = __syncthreads_and(all_keep);
+  const int any_commit = __syncthreads_or(committed);
   if (accepted && threadIdx.x == 0) accepted[b] = (uint8_t)acc;
+  if (p.min_commit && !any_commit && threadIdx.x == 0 && best_key != 0ull) {
+    // progress: nothing passed the threshold, so the most confident masked position commits
+    const int i = (int)(0xFFFFFFFFu - (uint32_t)(best_key & 0xFFFFFFFFull));
+    const int64_t row = (int64_t)b * R + (i - pos_offset);
+    decision[(int64_t)b * L + i] = DD_COMMIT;
+    new_tokens[(int64_t)b * L + i] = sampled ? st.sample_t[row] : st.argmax_t[row];
+  }
 }
 
 // Failure-detection self-test: wait on an mbarrier that nobody arrives on.
@@ -231,8 +268,8 @@ __global__ void selftest_wait_kernel(uint32_t limit) {
 
 cudaError_t launch_select_seeds(const float* entropy, int R, int pos_offset, const float* d_in,
                                 const float* d_out, const uint8_t* eligible, int B, int L, int k,
-                                int32_t* seeds, uint8_t* is_seed, float* score,
-                                cudaStream_t stream) {
+                                float min_score, int32_t* seeds, uint8_t* is_seed, float* score,
+                                int32_t* count, cudaStream_t stream) {
   const size_t smem = (size_t)L * sizeof(uint32_t);
   static thread_local int configured_for = -1;
   const DeviceInfo& dev = device_info();
@@ -244,7 +281,8 @@ cudaError_t launch_select_seeds(const float* entropy, int R, int pos_offset, con
     configured_for = dev.device;
   }
   select_seeds_kernel<<<B, kSelThreads, smem, stream>>>(entropy, R, pos_offset, d_in, d_out,
-                                                        eligible, L, k, seeds, is_seed, score);
+                                                        eligible, L, k, min_score, seeds, is_seed,
+                                                        score, count);
   return cudaGetLastError();
 }
 

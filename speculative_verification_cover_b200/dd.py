@@ -18,15 +18,16 @@ LIB_PATH = os.path.join(_HERE, "libdd.so")
 
 DD_OK, DD_ERR_INVALID_ARG, DD_ERR_UNSUPPORTED, DD_ERR_CUDA, DD_ERR_TIMEOUT = range(5)
 DD_F32, DD_BF16 = 0, 1
-POLICIES = {"trust": 0, "kl": 1, "conf": 2, "cover": 3, "coupled": 4}
-DD_NONE, DD_KEEP, DD_REPLACE, DD_REMASK = 0, 1, 2, 3
+POLICIES = {"trust": 0, "kl": 1, "conf": 2, "cover": 3, "coupled": 4, "kl_stochastic": 5}
+DD_NONE, DD_KEEP, DD_REPLACE, DD_REMASK, DD_COMMIT = 0, 1, 2, 3, 4
 DD_MASK_TOKEN = -1
 
 # Every symbol include/dd.h declares.
 EXPORTED = (
-    "dd_dualview_attention", "dd_dualview_attention_workspace_size", "dd_verify_logits",
+    "dd_dualview_attention", "dd_dualview_attention_ex", "dd_dualview_attention_workspace_size", "dd_verify_logits",
     "dd_verify_logits_workspace_size", "dd_verify_logits_static",
-    "dd_coupled_gumbel", "dd_select_seeds", "dd_decide", "dd_status_string",
+    "dd_coupled_gumbel", "dd_select_seeds", "dd_select_seeds_ex", "dd_decide",
+    "dd_status_string",
     "dd_get_device_error", "dd_set_spin_limit", "dd_selftest_bounded_wait",
     "dd_selftest_gumbel_screen",
 )
@@ -46,7 +47,9 @@ class _RowStats(ctypes.Structure):
 
 class _DecideParams(ctypes.Structure):
     _fields_ = [("policy", ctypes.c_int), ("tau_kl", ctypes.c_float),
-                ("tau_conf", ctypes.c_float), ("temperature", ctypes.c_float)]
+                ("tau_conf", ctypes.c_float), ("temperature", ctypes.c_float),
+                ("tau_commit", ctypes.c_float), ("min_commit", ctypes.c_int),
+                ("seed", ctypes.c_uint64), ("step", ctypes.c_uint64)]
 
 
 _lib = None
@@ -65,6 +68,8 @@ def lib():
                              ctypes.c_float, ctypes.c_size_t)
     L.dd_dualview_attention.argtypes = [P] * 8 + [I] * 5 + [F, I, I] + [P] * 5 + [SZ, P]
     L.dd_dualview_attention.restype = I
+    L.dd_dualview_attention_ex.argtypes = [P] * 8 + [I] * 5 + [F, I, I, I, F] + [P] * 5 + [SZ, P]
+    L.dd_dualview_attention_ex.restype = I
     L.dd_dualview_attention_workspace_size.argtypes = [I] * 5
     L.dd_dualview_attention_workspace_size.restype = SZ
     L.dd_verify_logits.argtypes = [P, P, I, I, I, I, I64, I, F, U64, U64,
@@ -79,6 +84,8 @@ def lib():
     L.dd_coupled_gumbel.restype = I
     L.dd_select_seeds.argtypes = [P, I, I, P, P, P, I, I, I, P, P, P, P]
     L.dd_select_seeds.restype = I
+    L.dd_select_seeds_ex.argtypes = [P, I, I, P, P, P, I, I, I, F, P, P, P, P, P]
+    L.dd_select_seeds_ex.restype = I
     L.dd_decide.argtypes = [ctypes.POINTER(_DecideParams), P, P, P, ctypes.POINTER(_RowStats),
                             I, I, I, I, P, P, P, P]
     L.dd_decide.restype = I
@@ -179,6 +186,23 @@ def dd_dualview_attention(q, k_cur, v_cur, k_prev, v_prev, is_seed, is_masked, i
     _check("dd_dualview_attention", st)
 
 
+def dd_dualview_attention_ex(q, k_cur, v_cur, k_prev, v_prev, is_seed, is_masked, is_new,
+                             out, lse, d_in=None, d_out=None, workspace=None, q_begin=0,
+                             accumulate_stats=False, stats_weight=1.0, softmax_scale=0.0,
+                             stream=None):
+    """One layer of a multi-layer pass with a prefix cache: query rows from q_begin on,
+    this layer's d_in / d_out weighted by stats_weight (see include/dd.h)."""
+    B, L, Hq, d = q.shape
+    Hkv = k_cur.shape[2]
+    nbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = lib().dd_dualview_attention_ex(
+        _ptr(q), _ptr(k_cur), _ptr(v_cur), _ptr(k_prev), _ptr(v_prev), _ptr(is_seed),
+        _ptr(is_masked), _ptr(is_new), B, L, Hq, Hkv, d, float(softmax_scale), _dtype_code(q),
+        int(q_begin), int(bool(accumulate_stats)), float(stats_weight), _ptr(out), _ptr(lse),
+        _ptr(d_in), _ptr(d_out), _ptr(workspace), nbytes, _stream(stream))
+    _check("dd_dualview_attention_ex", st)
+
+
 def dd_verify_logits_workspace_size(B, R, V, dtype) -> int:
     code = dtype if isinstance(dtype, int) else _dtype_code(torch.empty(0, dtype=dtype))
     return int(lib().dd_verify_logits_workspace_size(B, R, V, code))
@@ -248,15 +272,32 @@ def dd_select_seeds(entropy, pos_offset, d_in, d_out, eligible, seeds, is_seed=N
     _check("dd_select_seeds", st)
 
 
+def dd_select_seeds_ex(entropy, pos_offset, d_in, d_out, eligible, seeds, is_seed=None,
+                       score=None, count=None, min_score=float("-inf"), stream=None):
+    """dd_select_seeds with an adaptive size: only scores >= min_score compete;
+    count [B] int32 (optional) receives the number chosen per sequence."""
+    B, L = d_in.shape
+    R = entropy.shape[1] if entropy is not None else 0
+    k = seeds.shape[1] if seeds is not None else 0
+    st = lib().dd_select_seeds_ex(_ptr(entropy), R, int(pos_offset), _ptr(d_in), _ptr(d_out),
+                                  _ptr(eligible), B, L, k, float(min_score), _ptr(seeds),
+                                  _ptr(is_seed), _ptr(score), _ptr(count), _stream(stream))
+    _check("dd_select_seeds_ex", st)
+
+
 def dd_decide(policy, tokens, is_seed, eligible, stats: RowStats, pos_offset, decision,
-              new_tokens, accepted=None, tau_kl=0.5, tau_conf=0.9, temperature=0.0, stream=None):
+              new_tokens, accepted=None, tau_kl=0.5, tau_conf=0.9, temperature=0.0,
+              tau_commit=0.0, min_commit=0, seed=0, step=0, stream=None):
     """tokens [B,L] int32; stats from dd_verify_logits ([B,R]); decision [B,L] u8,
-    new_tokens [B,L] int32, accepted [B] u8 outputs."""
+    new_tokens [B,L] int32, accepted [B] u8 outputs. tau_commit > 0 turns on dynamic
+    threshold decoding of masked positions; seed / step key the draws of the
+    stochastic KL policy."""
     B, L = tokens.shape
     ref = stats.argmax_t if stats.argmax_t is not None else stats.sample_t
     R = ref.shape[1]
     p = _DecideParams(POLICIES[policy] if isinstance(policy, str) else int(policy),
-                      float(tau_kl), float(tau_conf), float(temperature))
+                      float(tau_kl), float(tau_conf), float(temperature), float(tau_commit),
+                      int(min_commit), int(seed) & (2**64 - 1), int(step) & (2**64 - 1))
     st = lib().dd_decide(ctypes.byref(p), _ptr(tokens), _ptr(is_seed), _ptr(eligible),
                          ctypes.byref(stats._c()), B, L, R, int(pos_offset), _ptr(decision),
                          _ptr(new_tokens), _ptr(accepted), _stream(stream))

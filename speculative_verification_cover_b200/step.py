@@ -1,7 +1,8 @@
 """One verification step over device-resident buffers, built on the C ABI.
 
 A step is the four library calls in order, on one stream:
-  1. dd_dualview_attention  -- dual-view attention (one layer) with d_in, d_out
+  1. dd_dualview_attention  -- dual-view attention (one layer, or each layer of a
+                               stack, optionally after a cached prefix) with d_in, d_out
   2. dd_verify_logits       -- per-row statistics and coupled samples
   3. dd_select_seeds        -- the next step's seed set from u, d_in, d_out
   4. dd_decide              -- KEEP / REPLACE / REMASK
@@ -17,16 +18,23 @@ from .workloads import WorkloadSpec
 
 INPUT_KEYS = ("q", "k_cur", "v_cur", "k_prev", "v_prev", "is_seed", "is_masked", "is_new",
               "eligible", "tokens", "logits_t", "logits_d")
-# Our kernels per step: mask preparation, attention pass 1, pass 2, head
-# reduction, vocabulary stream + merge, seed selection, decisions.
-KERNELS_PER_STEP = 8
+# Our kernels per step: per attention layer mask preparation, pass 1, pass 2 and
+# the head reduction; vocabulary stream + merge; seed selection; decisions.
+KERNELS_PER_LAYER = 4
+KERNELS_PER_STEP = KERNELS_PER_LAYER + 4  # one attention layer
 
 
 class VerifyStep:
     def __init__(self, spec: WorkloadSpec, inputs: dict, seed: int = 2024, step_index: int = 1,
-                 use_seeds: bool = True):
+                 use_seeds: bool = True, extra_layers=(), prefix_cache: bool = False):
+        """extra_layers: attention operands (q, k_cur, v_cur, k_prev, v_prev) of further
+        layers after the one in `inputs`; the step then runs every layer, averaging d_in
+        and d_out over them. prefix_cache: the prompt's K/V rows are a cache filled
+        once, so every layer computes the query rows after the prompt only."""
         self.spec = spec
         self.x = {k: inputs[k] for k in INPUT_KEYS}
+        self.extra_layers = list(extra_layers)
+        self.q_begin = spec.prompt if prefix_cache else 0
         dev = self.x["q"].device
         B, L, Hq, Hkv, d, R = spec.B, spec.L, spec.Hq, spec.Hkv, spec.d, spec.R
         self.seed, self.step_index = seed, step_index
@@ -51,13 +59,23 @@ class VerifyStep:
         self.graphs = None
         self.side = None
 
+    @property
+    def n_layers(self):
+        return 1 + len(self.extra_layers)
+
+    @property
+    def kernels_per_step(self):
+        return KERNELS_PER_LAYER * self.n_layers + 4
+
     # --- the four calls
     def attention(self):
-        x = self.x
-        dd.dd_dualview_attention(
-            x["q"], x["k_cur"], x["v_cur"], x["k_prev"] if self.use_seeds else None,
-            x["v_prev"] if self.use_seeds else None, x["is_seed"] if self.use_seeds else None,
-            x["is_masked"], x["is_new"], self.out, self.lse, self.d_in, self.d_out, self.ws)
+        x, n = self.x, self.n_layers
+        for li, y in enumerate([x] + self.extra_layers):
+            dd.dd_dualview_attention_ex(
+                y["q"], y["k_cur"], y["v_cur"], y["k_prev"] if self.use_seeds else None,
+                y["v_prev"] if self.use_seeds else None, x["is_seed"] if self.use_seeds else None,
+                x["is_masked"], x["is_new"], self.out, self.lse, self.d_in, self.d_out, self.ws,
+                q_begin=self.q_begin, accumulate_stats=li > 0, stats_weight=1.0 / n)
 
     def verify(self):
         s = self.spec

@@ -251,3 +251,91 @@ def random_logit_rows(n: int, V: int, gen: torch.Generator, logit_std=3.0, peak=
                             dtype={torch.float32: "f32", torch.bfloat16: "bf16"}[dtype])
     lt, ld, pk = _logits(spec, gen, torch.device(device))
     return lt[0], ld[0], pk[0]
+
+
+def layer_operands(spec: WorkloadSpec, device="cpu", seed: int = 0, n_layers: int = 1) -> list:
+    """Attention operands (q, k_cur, v_cur, k_prev, v_prev) of n_layers further layers of
+    one verification step, with the distributions of spec (a separate seeded stream per
+    call). Sequences share the position masks of make_inputs; only the operands differ
+    from layer to layer."""
+    device = torch.device(device)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    is_new = torch.zeros(spec.B, spec.L, dtype=torch.uint8, device=device)
+    out = []
+    for _ in range(n_layers):
+        q, k, v, kp, vp = _attention_operands(spec, gen, device, is_new)
+        out.append(dict(q=q, k_cur=k, v_cur=v, k_prev=kp, v_prev=vp))
+    return out
+
+
+class DecodeDynamics:
+    """Seeded synthetic stand-in for the models of a multi-step decode: it draws, from
+    the current token assignment, the attention operands and the verifier / drafter
+    logits of the next verification step. It holds none of the method's arithmetic.
+
+    * Every sequence has a hidden target token per generated position.
+    * Q / K / V rows are looked up by the position's current token (a table of
+      `table` rows, [MASK] its own row) plus a positional row, so a token that
+      changes changes its K / V, and the previous step's K / V act as a cache.
+    * Verifier logits of a generated position: N(0, logit_std) plus a peak of
+      height ln V + 4 + 8 c on the target with probability 0.5 + 0.45 c, else on a
+      fixed confusable wrong token, where c is the fraction of the sequence's
+      generated positions that currently hold their target (more correct context,
+      a more confident and more accurate verifier; the ln V term makes the peak's
+      probability independent of the vocabulary size). Drafter = verifier +
+      N(0, drafter_std).
+    """
+
+    def __init__(self, spec: WorkloadSpec, device="cpu", seed: int = 0, table: int = 4096):
+        device = torch.device(device)
+        self.spec, self.device, self.table = spec, device, table
+        self.gen = torch.Generator(device=device)
+        self.gen.manual_seed(seed)
+        g, B, L, V = self.gen, spec.B, spec.L, spec.V
+        dt = _torch_dtype(spec.dtype)
+        self.dtype = dt
+        std = spec.qkv_std
+        self.Eq = _randn(g, (table + 1, spec.Hq, spec.d), std, device)
+        self.Ek = _randn(g, (table + 1, spec.Hkv, spec.d), std, device)
+        self.Ev = _randn(g, (table + 1, spec.Hkv, spec.d), std, device)
+        self.Pq = _randn(g, (L, spec.Hq, spec.d), std, device)
+        self.Pk = _randn(g, (L, spec.Hkv, spec.d), std, device)
+        self.Pv = _randn(g, (L, spec.Hkv, spec.d), std, device)
+        self.target = torch.randint(0, V, (B, L), generator=g, device=device)
+        self.wrong = (self.target + 1 + torch.randint(0, V - 1, (B, L), generator=g,
+                                                      device=device)) % V
+        prompt_tok = torch.randint(0, V, (B, spec.prompt), generator=g, device=device)
+        self.initial = torch.full((B, L), MASK_TOKEN, dtype=torch.int32, device=device)
+        self.initial[:, :spec.prompt] = prompt_tok.to(torch.int32)
+        self.target[:, :spec.prompt] = prompt_tok
+
+    def _rows(self, tokens):
+        return torch.where(tokens < 0, torch.full_like(tokens, self.table),
+                           tokens.long() % self.table)
+
+    def operands(self, tokens, masked_view=None):
+        """q, k, v [B, L, H, d] for `tokens`; positions in masked_view (u8 [B, L], or None)
+        are looked up as [MASK] (the verification view of seeds)."""
+        rows = self._rows(tokens)
+        if masked_view is not None:
+            rows = torch.where(masked_view.bool(), torch.full_like(rows, self.table), rows)
+        q = self.Eq[rows] + self.Pq
+        k = self.Ek[rows] + self.Pk
+        v = self.Ev[rows] + self.Pv
+        return [x.to(self.dtype).contiguous() for x in (q, k, v)]
+
+    def logits(self, tokens):
+        """Verifier and drafter logits [B, R, V] of the generated rows for `tokens`."""
+        s, g, dev = self.spec, self.gen, self.device
+        B, R, V, P = s.B, s.R, s.V, s.prompt
+        correct = (tokens[:, P:].long() == self.target[:, P:]).float().mean(dim=1)  # [B]
+        c = correct[:, None]
+        right = torch.rand(B, R, generator=g, device=dev) < (0.5 + 0.45 * c)
+        peak_tok = torch.where(right, self.target[:, P:], self.wrong[:, P:])
+        x = _randn(g, (B, R, V), s.logit_std, dev)
+        height = math.log(V) + 4.0 + 8.0 * c
+        x.scatter_add_(2, peak_tok[..., None], height.expand(B, R)[..., None])
+        lt = x.to(self.dtype)
+        x += _randn(g, (B, R, V), s.drafter_std, dev)
+        return lt, x.to(self.dtype)

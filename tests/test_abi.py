@@ -165,3 +165,23 @@ def test_attention_ex_validation(lib):
     assert ex(weight=float("nan")) == dd.DD_ERR_INVALID_ARG
     assert ex(weight=float("inf")) == dd.DD_ERR_INVALID_ARG
     assert ex(L=0) == dd.DD_ERR_INVALID_ARG
+
+
+def test_select_ex_and_decide_extension_validation(lib):
+    nan = float("nan")
+    assert lib.dd_select_seeds_ex(FAKE, 4, 0, FAKE, FAKE, FAKE, 1, 8, 2, nan, FAKE, None, None,
+                                  None, None) == dd.DD_ERR_INVALID_ARG
+    stats = dd._RowStats()
+    stats.argmax_t = FAKE
+    stats.kl_dt = FAKE
+    # the stochastic KL rule needs a positive threshold
+    p = dd._DecideParams(5, 0.0, 0.9, 0.0, 0.0, 0, 1, 2)
+    assert lib.dd_decide(ctypes.byref(p), FAKE, FAKE, FAKE, ctypes.byref(stats), 1, 8, 4, 0,
+                         FAKE, FAKE, None, None) == dd.DD_ERR_INVALID_ARG
+    # min_commit is 0 or 1; commit needs p_sample_t
+    p = dd._DecideParams(0, 0.5, 0.9, 0.0, 0.5, 2, 0, 0)
+    assert lib.dd_decide(ctypes.byref(p), FAKE, FAKE, FAKE, ctypes.byref(stats), 1, 8, 4, 0,
+                         FAKE, FAKE, None, None) == dd.DD_ERR_INVALID_ARG
+    p = dd._DecideParams(0, 0.5, 0.9, 0.0, 0.5, 1, 0, 0)
+    assert lib.dd_decide(ctypes.byref(p), FAKE, FAKE, FAKE, ctypes.byref(stats), 1, 8, 4, 0,
+                         FAKE, FAKE, None, None) == dd.DD_ERR_INVALID_ARG

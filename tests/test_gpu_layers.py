@@ -49,7 +49,8 @@ def _check(x, layers, outs, lses, d_in, d_out, q_begin, b, heads, tol, with_seed
                                          PA.npi(x["is_new"][b]), q_begin=q_begin)
     for li in range(len(layers)):
         PA.assert_close(f"out[{li}]", f(outs[li][b, q_begin:])[:, heads], wo[li][:, heads], 0, tol)
-        PA.assert_close(f"lse[{li}]", f(lses[li][b, :, q_begin:])[heads], wl[li][heads], 1e-5, 1e-4)
+        PA.assert_close(f"lse[{li}]", f(lses[li][b, :, q_begin:])[heads], wl[li][heads],
+                        PA.STAT_RTOL, PA.STAT_ATOL)
         assert bool((outs[li][b, :q_begin] == 3.0).all()), "prefix rows of out were written"
         assert bool((lses[li][b, :, :q_begin] == 5.0).all()), "prefix rows of lse were written"
     PA.assert_close("d_in", f(d_in[b]), wdin, PA.MASS_RTOL, PA.MASS_ATOL)

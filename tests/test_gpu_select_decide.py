@@ -4,6 +4,7 @@ import pytest
 import torch
 
 from speculative_verification_cover_b200 import dd
+from oracle import decide as OD
 from oracle import seeds as OS
 from tests import parity as PA
 
@@ -127,3 +128,93 @@ def test_decide_matches_oracle(policy, T):
         assert np.array_equal(PA.npi(newt[b]), wt.astype(np.int64)), (policy, b)
         assert int(acc[b]) == wa, (policy, b)
         assert int(near.sum()) <= 2  # positions within 1e-4 of a threshold: counted
+
+
+@pytest.mark.parametrize("min_score", [-1.0, 2.0, 6.5, 100.0])
+def test_adaptive_seed_set_matches_oracle(min_score):
+    rng = np.random.default_rng(int(min_score * 10) + 77)
+    B, L, R, off, k = 3, 700, 560, 140, 48
+    entropy = rng.random((B, R)) * 5
+    d_in = rng.random((B, L)) * 3
+    d_out = rng.random((B, L))
+    elig = (rng.random((B, L)) < 0.6).astype(np.uint8)
+    t = lambda a, dt=torch.float32: torch.tensor(a, dtype=dt, device="cuda")
+    seeds = torch.full((B, k), -5, dtype=torch.int32, device="cuda")
+    is_seed = torch.full((B, L), 9, dtype=torch.uint8, device="cuda")
+    score = torch.empty(B, L, device="cuda")
+    count = torch.full((B,), -1, dtype=torch.int32, device="cuda")
+    dd.dd_select_seeds_ex(t(entropy), off, t(d_in), t(d_out), t(elig, torch.uint8), seeds,
+                          is_seed, score, count, min_score=min_score)
+    torch.cuda.synchronize()
+    for b in range(B):
+        u32 = np.zeros(L, np.float32)
+        u32[off:off + R] = np.float32(entropy[b])
+        el = elig[b].astype(bool).copy()
+        el[:off] = False
+        el[off + R:] = False
+        s32 = (u32 * (np.float32(1) + np.float32(d_in[b]))) / (np.float32(1) + np.float32(d_out[b]))
+        sc = np.where(el, s32.astype(np.float64), -np.inf)
+        want, want_is = OS.select(sc, k, float(np.float32(min_score)))
+        assert np.array_equal(PA.npi(seeds[b]), want), b
+        assert np.array_equal(PA.npi(is_seed[b]), want_is.astype(np.int64)), b
+        assert int(count[b]) == int((want >= 0).sum())
+
+
+def _random_stats(rng, B, R, V):
+    st = dict(
+        lse_t=rng.random((B, R)), lse_d=rng.random((B, R)), conf_t=rng.random((B, R)),
+        p_sample_t=rng.random((B, R)), entropy_t=rng.random((B, R)), kl_dt=rng.random((B, R)),
+        argmax_t=rng.integers(0, V, (B, R)), argmax_d=rng.integers(0, V, (B, R)),
+        sample_t=rng.integers(0, V, (B, R)), sample_d=rng.integers(0, V, (B, R)))
+    return st
+
+
+def _stats_dev(st):
+    return dd.RowStats(**{k: torch.tensor(v, dtype=torch.float32 if v.dtype.kind == "f"
+                                          else torch.int32, device="cuda")
+                          for k, v in st.items()})
+
+
+@pytest.mark.parametrize("policy,T,tau_commit,min_commit", [
+    ("kl_stochastic", 0.0, 0.0, 0), ("kl_stochastic", 0.8, 0.0, 0),
+    ("kl_stochastic", 0.0, 0.7, 1), ("cover", 0.0, 0.8, 0), ("coupled", 0.8, 0.8, 1),
+    ("trust", 0.0, 2.0, 1),      # nothing passes: the progress rule commits one per sequence
+    ("trust", 0.8, 2.0, 0),      # nothing passes and no progress rule: no commit
+])
+def test_decide_stochastic_and_commit_match_oracle(policy, T, tau_commit, min_commit):
+    rng = np.random.default_rng(hash((policy, T, tau_commit, min_commit)) % 2**32)
+    B, L, R, off, V = 4, 300, 240, 60, 20
+    tokens = rng.integers(0, V, (B, L)).astype(np.int32)
+    masked = rng.random((B, L)) < 0.3
+    tokens[masked] = -1
+    elig = (~masked).astype(np.uint8)
+    elig[:, :off] = 0
+    is_seed = ((rng.random((B, L)) < 0.2) & (elig == 1)).astype(np.uint8)
+    st = _random_stats(rng, B, R, V)
+    st["p_sample_t"][0, :5] = 0.625  # exact ties for the progress rule (binary fraction)
+    seed, step = 0x1234ABCD5678, 9
+    dec = torch.empty(B, L, dtype=torch.uint8, device="cuda")
+    newt = torch.empty(B, L, dtype=torch.int32, device="cuda")
+    acc = torch.empty(B, dtype=torch.uint8, device="cuda")
+    tau_kl = 0.5
+    dd.dd_decide(policy, torch.tensor(tokens, device="cuda"), torch.tensor(is_seed, device="cuda"),
+                 torch.tensor(elig, device="cuda"), _stats_dev(st), off, dec, newt, acc,
+                 tau_kl=tau_kl, tau_conf=0.6, temperature=T, tau_commit=tau_commit,
+                 min_commit=min_commit, seed=seed, step=step)
+    torch.cuda.synchronize()
+    f32 = lambda v: float(np.float32(v))
+    commits = 0
+    for b in range(B):
+        rows = {k: np.float32(v[b]).astype(np.float64) if v.dtype.kind == "f" else v[b]
+                for k, v in st.items()}
+        rows["margin_t"] = np.full(R, np.inf)
+        rows["margin_d"] = np.full(R, np.inf)
+        wd, wt, wa, near = OD.decide(policy, tokens[b], is_seed[b], elig[b], rows, off, R, T,
+                                     f32(tau_kl), f32(0.6), PA.TIE_EPS, f32(tau_commit),
+                                     min_commit, seed, step, b)
+        assert np.array_equal(PA.npi(dec[b]), wd.astype(np.int64)), (policy, b)
+        assert np.array_equal(PA.npi(newt[b]), wt.astype(np.int64)), (policy, b)
+        assert int(acc[b]) == wa, (policy, b)
+        commits += int((wd == OD.COMMIT).sum())
+    if tau_commit == 2.0:
+        assert commits == (B if min_commit else 0)

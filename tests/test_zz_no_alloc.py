@@ -45,8 +45,14 @@ def test_static_scratch_matches_workspace_variant_two_calls_in_a_row():
     cases = [  # (seed, B, R, V, dtype, temperature, pos_offset)
         (11, 3, 40, 32000, torch.bfloat16, 0.0, 5),
         (12, 2, 64, 50257, torch.bfloat16, 1.0, 0),
+        (13, 4, 64, 50257, torch.float32, 0.7, 3),     # fp32 logits
+        (14, 16, 2000, 64, torch.bfloat16, 1.0, 0),    # scratch just under the 4 MiB array
     ]
     for seed, B, R, V, dtype, T, off in cases:
+        need = dd.dd_verify_logits_workspace_size(B, R, V, dtype)
+        assert need <= 4 << 20
+        if seed == 14:
+            assert need > 0.95 * (4 << 20)  # the array is nearly full
         V_pad = (V + 7) // 8 * 8
         lt_full, lm_full = _inputs(seed, B, R, V_pad, dtype)
         lt, lm = lt_full[..., :V], lm_full[..., :V]
