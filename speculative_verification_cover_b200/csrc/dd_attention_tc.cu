@@ -696,27 +696,19 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // 4-D map over a [B, L, H, D] bf16 tensor, dims innermost first {D, H, L, B};
 // box = 64 head-dim elements (128 bytes) x 1 head x 128 positions x 1 sequence.
-bool make_map(CUtensorMap* map, const void* base, int D, int H, int L, int B) {
+bool make_map(CUtensorMap* map, const void* base, int D, int H, int L, int B, int box_rows = 128) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)L, (cuuint64_t)B};
   cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)L * H * D * 2};
-  cuuint32_t box[4] = {64, 1, 128, 1};
+  cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D>
-cudaError_t launch_p1(const AttnArgs& a, bool pass2, cudaStream_t stream) {
-  CUtensorMap tq, tk, tv;
-  // without seeds the drafting view is the current input itself
-  const void* kv = a.is_seed ? a.k_view : a.k_cur;
-  const void* vv = a.is_seed ? a.v_view : a.v_cur;
-  if (!make_map(&tq, a.q, D, a.Hq, a.L, a.B) || !make_map(&tk, kv, D, a.Hkv, a.L, a.B) ||
-      !make_map(&tv, vv, D, a.Hkv, a.L, a.B))
-    return cudaErrorInvalidValue;
+P1Params p1_params(const AttnArgs& a, bool pass2) {
   P1Params p;
   p.q = static_cast<const __nv_bfloat16*>(a.q);
   p.k_cur = static_cast<const __nv_bfloat16*>(a.k_cur);
@@ -737,6 +729,19 @@ cudaError_t launch_p1(const AttnArgs& a, bool pass2, cudaStream_t stream) {
   p.q_m = pass2 ? static_cast<__nv_bfloat16*>(a.q_m) : nullptr;
   p.lse2_m = a.lse2_m;
   p.spin = spin_limit();
+  return p;
+}
+
+template <int D>
+cudaError_t launch_p1(const AttnArgs& a, bool pass2, cudaStream_t stream) {
+  CUtensorMap tq, tk, tv;
+  // without seeds the drafting view is the current input itself
+  const void* kv = a.is_seed ? a.k_view : a.k_cur;
+  const void* vv = a.is_seed ? a.v_view : a.v_cur;
+  if (!make_map(&tq, a.q, D, a.Hq, a.L, a.B) || !make_map(&tk, kv, D, a.Hkv, a.L, a.B) ||
+      !make_map(&tv, vv, D, a.Hkv, a.L, a.B))
+    return cudaErrorInvalidValue;
+  const P1Params p = p1_params(a, pass2);
   const DeviceInfo& di = device_info();
   const int smem = P1Layout<D>::kBytes + 1024;
   static int configured[64] = {};
@@ -783,12 +788,23 @@ cudaError_t launch_p2(const AttnArgs& a, cudaStream_t stream) {
 
 }  // namespace
 
+template <int D>
+cudaError_t launch_p1x2(const AttnArgs& a, bool pass2, cudaStream_t stream);
+
 // Both passes on tensor cores. d_in partials are per kv head ([B, Hkv, L]).
+// Pass 1 takes two query tiles per CTA where that still gives every SM a few CTAs
+// (the tiles then share K / V and the tensor core alternates between them), one
+// tile per CTA otherwise (short sequences, where a 256-row CTA would leave SMs idle).
 cudaError_t launch_attention_tc(const AttnArgs& a, cudaStream_t stream, bool* handled,
                                 int* din_slices) {
   *handled = true;
   const bool pass2 = a.d_in != nullptr && a.is_masked != nullptr;
-  cudaError_t err = a.d == 64 ? launch_p1<64>(a, pass2, stream) : launch_p1<128>(a, pass2, stream);
+  const int64_t ctas2 = (int64_t)((a.L - a.q_begin + 2 * kBM - 1) / (2 * kBM)) * a.Hq * a.B;
+  const bool two = ctas2 >= 2 * (int64_t)device_info().sm_count;
+  cudaError_t err = two ? (a.d == 64 ? launch_p1x2<64>(a, pass2, stream)
+                                     : launch_p1x2<128>(a, pass2, stream))
+                        : (a.d == 64 ? launch_p1<64>(a, pass2, stream)
+                                     : launch_p1<128>(a, pass2, stream));
   if (err != cudaSuccess) return err;
   if (pass2) {
     err = a.d == 64 ? launch_p2<64>(a, stream) : launch_p2<128>(a, stream);

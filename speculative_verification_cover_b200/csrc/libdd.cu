@@ -4,5 +4,6 @@
 #include "dd_verify.cu"
 #include "dd_attention.cu"
 #include "dd_attention_tc.cu"
+#include "dd_attention_tc2.cu"
 #include "dd_select.cu"
 #include "dd_static.cu"
