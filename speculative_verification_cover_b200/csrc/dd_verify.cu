@@ -171,7 +171,7 @@ struct Unpack<float> {
 // word, its exact fp32 Gumbel value and its two scores. Entries are kept by exact
 // vocabulary index (encoded -1 - v), ties going to the lower index.
 constexpr int kQueueCap = 80;    // vectors per warp
-constexpr int kQueueDrain = 4;   // evaluate once this many vectors are queued
+constexpr int kQueueDrain = 16;  // evaluate once this many vectors are queued
 
 struct NoiseQueue {
   int v[kQueueCap];             // first vocabulary index of the vector
@@ -209,9 +209,16 @@ __device__ __forceinline__ void exact_entry(Acc& a, int v, float l, float m, con
   keep_best(a.bd, a.vbd, fmaf(m, invT, g), v);
 }
 
+// The best exact coupled scores any lane in `act` holds (the screen's thresholds).
+__device__ __forceinline__ void warp_thresholds(const Acc& a, unsigned act, float& tht,
+                                                float& thd) {
+  tht = ordered_to_float(__reduce_max_sync(act, float_to_ordered(a.bt)));
+  thd = ordered_to_float(__reduce_max_sync(act, float_to_ordered(a.bd)));
+}
+
 // Every queued entry, spread over the lanes in `act`; empties the queue.
 template <typename T>
-__device__ __noinline__ void drain_queue(Acc& a, NoiseQueue* q, int& qn, unsigned act,
+__device__ __forceinline__ void drain_queue(Acc& a, NoiseQueue* q, int& qn, unsigned act,
                                          const PhiloxRow& pr, NoiseKey key, float invT) {
   constexpr int VEC = Unpack<T>::N;
   __syncwarp(act);  // the pushes are visible
@@ -229,7 +236,8 @@ __device__ __noinline__ void drain_queue(Acc& a, NoiseQueue* q, int& qn, unsigne
 template <typename T, bool SAMPLE, int NV>
 __device__ __forceinline__ void fold(Acc& a, const uint4 (&lw)[NV], const uint4 (&mw)[NV],
                                      const int (&v0)[NV], const PhiloxRow& pr,
-                                     const NoiseKey& key, float invT, NoiseQueue* q, int& qn) {
+                                     const NoiseKey& key, float invT, NoiseQueue* q, int& qn,
+                                     float& tht, float& thd) {
   constexpr int VEC = Unpack<T>::N, NP = VEC / 2;
   float xm[NV], ym[NV];  // per-vector maxima of l and m
 #pragma unroll
@@ -289,10 +297,11 @@ __device__ __forceinline__ void fold(Acc& a, const uint4 (&lw)[NV], const uint4 
       a.skd = __ffma2_rn(ed, __ffma2_rn(lp, neg1, mp), a.skd);
     }
   // --- coupled Gumbel-max samples (same noise for both).
-  // Screening, per 16-byte vector: thr_t / thr_d are the best exact scores any lane
-  // of the warp holds for this row (all lanes work on one row, and every vector of
+  // Screening, per 16-byte vector: tht / thd are the best exact scores any lane of
+  // the warp holds for this row (all lanes work on one row, and every vector of
   // this fold lies above every entry evaluated so far, so such a score wins a tie
-  // against any entry here). An entry with noise g scores at most x_max / T + g; it
+  // against any entry here). They change only when exact scores are added, so the
+  // caller keeps them and they are refreshed after each evaluation of the queue. An entry with noise g scores at most x_max / T + g; it
   // can only matter if g exceeds G = min over the two matrices of (thr - x_max / T),
   // minus a rounding slack. If G >= kGumbelMax no noise value can do that and the
   // vector's generator words are not even drawn; otherwise the words are drawn and
@@ -301,8 +310,6 @@ __device__ __forceinline__ void fold(Acc& a, const uint4 (&lw)[NV], const uint4 
   // exactly the fp32 noise and scores the unscreened pass would compute.
   if constexpr (SAMPLE) {
     const unsigned act = __activemask();
-    const float tht = ordered_to_float(__reduce_max_sync(act, float_to_ordered(a.bt)));
-    const float thd = ordered_to_float(__reduce_max_sync(act, float_to_ordered(a.bd)));
     // slack for the fp32 rounding of thr - x/T (about 1e-7 relative)
     const float slt = fmaf(fabsf(tht), 1e-5f, 1e-5f), sld = fmaf(fabsf(thd), 1e-5f, 1e-5f);
     const float is = invT * 1e-5f;
@@ -337,7 +344,10 @@ __device__ __forceinline__ void fold(Acc& a, const uint4 (&lw)[NV], const uint4 
         qn += __popc(bal);
       }
     }
-    if (qn >= kQueueDrain) drain_queue<T>(a, q, qn, act, pr, key, invT);
+    if (qn >= kQueueDrain) {
+      drain_queue<T>(a, q, qn, act, pr, key, invT);
+      warp_thresholds(a, act, tht, thd);
+    }
   }
 }
 
@@ -639,6 +649,7 @@ verify_stream_kernel(const VerifyArgs a) {
     };
     // per-row parts of the noise generator (only used when sampling)
     const PhiloxRow pr = philox_row((uint32_t)pos, (uint32_t)b, a.key.step, a.key.k0, a.key.k1);
+    float tht = -INFINITY, thd = -INFINITY;  // the screen's thresholds (warp-uniform)
     // both vectors of a half-step in one fold where both exist (one warp-wide
     // screening threshold per pair), else the one that does
     auto fold2 = [&](int bs, const uint4 (&l)[2], const uint4 (&m)[2]) {
@@ -648,7 +659,7 @@ verify_stream_kernel(const VerifyArgs a) {
         // never fold (and push) at the same time.
         if (__all_sync(__activemask(), bs + kVThreads < vlim)) {
           const int vv[2] = {bs * VEC, (bs + kVThreads) * VEC};
-          fold<T, SAMPLE, 2>(acc, l, m, vv, pr, a.key, a.invT, q, qn);
+          fold<T, SAMPLE, 2>(acc, l, m, vv, pr, a.key, a.invT, q, qn, tht, thd);
           return;
         }
       }
@@ -658,7 +669,7 @@ verify_stream_kernel(const VerifyArgs a) {
         if (idx < vlim) {
           const uint4 l1[1] = {l[k]}, m1[1] = {m[k]};
           const int vv[1] = {idx * VEC};
-          fold<T, SAMPLE, 1>(acc, l1, m1, vv, pr, a.key, a.invT, q, qn);
+          fold<T, SAMPLE, 1>(acc, l1, m1, vv, pr, a.key, a.invT, q, qn, tht, thd);
         }
       }
     };
@@ -681,6 +692,7 @@ verify_stream_kernel(const VerifyArgs a) {
           keep_best(acc.bt, acc.vbt, fmaf(vec_entry<T>(la[0], e), a.invT, g), v + e);
           keep_best(acc.bd, acc.vbd, fmaf(vec_entry<T>(ma[0], e), a.invT, g), v + e);
         }
+        if constexpr (SAMPLE) warp_thresholds(acc, __activemask(), tht, thd);
       }
       fold2(base, la, ma);
       ld2(base + 2 * kStep, la, ma);
