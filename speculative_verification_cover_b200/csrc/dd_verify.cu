@@ -167,9 +167,10 @@ struct Unpack<float> {
 // A lane whose 16-byte vector passes the noise screen does not evaluate it on its
 // own (that would hold the whole warp for the few lanes that need it); it pushes
 // the vector into its warp's queue in shared memory, and once a few vectors are
-// queued every lane of the warp takes one queued entry at a time: its generator
-// word, its exact fp32 Gumbel value and its two scores. Entries are kept by exact
-// vocabulary index (encoded -1 - v), ties going to the lower index.
+// queued every lane of the warp takes one generator counter (four consecutive
+// entries) at a time: the words, their exact fp32 Gumbel values and the scores.
+// Entries are kept by exact vocabulary index (encoded -1 - v), ties going to the
+// lower index.
 constexpr int kQueueCap = 80;    // vectors per warp
 constexpr int kQueueDrain = 16;  // evaluate once this many vectors are queued
 
@@ -196,19 +197,6 @@ __device__ __forceinline__ float vec_entry(const uint4& u, int e) {
   }
 }
 
-__device__ __forceinline__ uint32_t pick_word(const PhiloxOut& o, int i) {
-  return i == 0 ? o.w[0] : i == 1 ? o.w[1] : i == 2 ? o.w[2] : o.w[3];
-}
-
-// The exact coupled scores of entry v (logits l, m) into a lane's state.
-__device__ __forceinline__ void exact_entry(Acc& a, int v, float l, float m, const PhiloxRow& pr,
-                                            const NoiseKey& key, float invT) {
-  const PhiloxOut o = philox_row_counter(pr, (uint32_t)(v >> 2), key.k0, key.k1);
-  const float g = gumbel_from_word(pick_word(o, v & 3));
-  keep_best(a.bt, a.vbt, fmaf(l, invT, g), v);
-  keep_best(a.bd, a.vbd, fmaf(m, invT, g), v);
-}
-
 // The best exact coupled scores any lane in `act` holds (the screen's thresholds).
 __device__ __forceinline__ void warp_thresholds(const Acc& a, unsigned act, float& tht,
                                                 float& thd) {
@@ -224,10 +212,19 @@ __device__ __forceinline__ void drain_queue(Acc& a, NoiseQueue* q, int& qn, unsi
   __syncwarp(act);  // the pushes are visible
   const int lane = threadIdx.x & 31;
   const int nact = __popc(act), rank = __popc(act & ((1u << lane) - 1u));
-  for (int i = rank; i < qn * VEC; i += nact) {
-    const int s = i / VEC, e = i % VEC;
-    exact_entry(a, q->v[s] + e, vec_entry<T>(q->l[s], e), vec_entry<T>(q->m[s], e), pr, key,
-                invT);
+  // one generator counter (four consecutive entries) per lane and round
+  constexpr int NC = VEC / 4;  // counters per 16-byte vector
+  for (int i = rank; i < qn * NC; i += nact) {
+    const int s = i / NC, c = i % NC;
+    const int v = q->v[s] + 4 * c;
+    const uint4 lw = q->l[s], mw = q->m[s];
+    const PhiloxOut o = philox_row_counter(pr, (uint32_t)(v >> 2), key.k0, key.k1);
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const float g = gumbel_from_word(o.w[w]);
+      keep_best(a.bt, a.vbt, fmaf(vec_entry<T>(lw, 4 * c + w), invT, g), v + w);
+      keep_best(a.bd, a.vbd, fmaf(vec_entry<T>(mw, 4 * c + w), invT, g), v + w);
+    }
   }
   __syncwarp(act);  // every lane is done reading before the queue is reused
   qn = 0;
