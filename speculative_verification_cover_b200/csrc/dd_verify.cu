@@ -204,6 +204,22 @@ __device__ __forceinline__ void warp_thresholds(const Acc& a, unsigned act, floa
   thd = ordered_to_float(__reduce_max_sync(act, float_to_ordered(a.bd)));
 }
 
+// The warp's thresholds, raised to the CTA-wide best (every warp of a CTA works on the
+// same row piece). A threshold from any entry of the row keeps the screen exact: a
+// screened-out entry scores strictly below it (the slack), so it cannot be sampled.
+__device__ __forceinline__ void publish_thresholds(const Acc& a, unsigned act, float& tht,
+                                                   float& thd, int* cta_thr) {
+  warp_thresholds(a, act, tht, thd);
+  int ot = 0, od = 0;
+  const int lead = __ffs(act) - 1;
+  if ((int)(threadIdx.x & 31) == lead) {
+    ot = atomicMax(&cta_thr[0], float_to_ordered(tht));
+    od = atomicMax(&cta_thr[1], float_to_ordered(thd));
+  }
+  tht = fmaxf(tht, ordered_to_float(__shfl_sync(act, ot, lead)));
+  thd = fmaxf(thd, ordered_to_float(__shfl_sync(act, od, lead)));
+}
+
 // Every queued entry, spread over the lanes in `act`; empties the queue.
 template <typename T>
 __device__ __forceinline__ void drain_queue(Acc& a, NoiseQueue* q, int& qn, unsigned act,
@@ -234,7 +250,7 @@ template <typename T, bool SAMPLE, int NV>
 __device__ __forceinline__ void fold(Acc& a, const uint4 (&lw)[NV], const uint4 (&mw)[NV],
                                      const int (&v0)[NV], const PhiloxRow& pr,
                                      const NoiseKey& key, float invT, NoiseQueue* q, int& qn,
-                                     float& tht, float& thd) {
+                                     float& tht, float& thd, int* cta_thr) {
   constexpr int VEC = Unpack<T>::N, NP = VEC / 2;
   float xm[NV], ym[NV];  // per-vector maxima of l and m
 #pragma unroll
@@ -307,6 +323,9 @@ __device__ __forceinline__ void fold(Acc& a, const uint4 (&lw)[NV], const uint4 
   // exactly the fp32 noise and scores the unscreened pass would compute.
   if constexpr (SAMPLE) {
     const unsigned act = __activemask();
+    // the best the CTA's other warps have published for this row
+    tht = fmaxf(tht, ordered_to_float(*(volatile int*)&cta_thr[0]));
+    thd = fmaxf(thd, ordered_to_float(*(volatile int*)&cta_thr[1]));
     // slack for the fp32 rounding of thr - x/T (about 1e-7 relative)
     const float slt = fmaf(fabsf(tht), 1e-5f, 1e-5f), sld = fmaf(fabsf(thd), 1e-5f, 1e-5f);
     const float is = invT * 1e-5f;
@@ -343,7 +362,7 @@ __device__ __forceinline__ void fold(Acc& a, const uint4 (&lw)[NV], const uint4 
     }
     if (qn >= kQueueDrain) {
       drain_queue<T>(a, q, qn, act, pr, key, invT);
-      warp_thresholds(a, act, tht, thd);
+      publish_thresholds(a, act, tht, thd, cta_thr);
     }
   }
 }
@@ -586,9 +605,14 @@ verify_stream_kernel(const VerifyArgs a) {
   init(acc);
   // sampling: this warp's queue of vectors awaiting exact noise (see drain_queue)
   NoiseQueue* q = nullptr;
+  int* cta_thr = nullptr;  // the CTA's best exact scores of the current row (ordered ints)
   if constexpr (SAMPLE) {
     __shared__ NoiseQueue queues[kVThreads / 32];
+    __shared__ int thr_s[2];
     q = &queues[cw];
+    cta_thr = thr_s;
+    if (ct == 0) thr_s[0] = thr_s[1] = float_to_ordered(-INFINITY);
+    __syncthreads();
   }
   int qn = 0;
   auto flush = [&](int64_t row, Partial p) {
@@ -617,6 +641,8 @@ verify_stream_kernel(const VerifyArgs a) {
         const int64_t slot = c - a.split.cta_of(row * spr);
         a.parts[row * a.maxparts + slot] = r;
       }
+      // every warp is past the row: its thresholds start over for the next one
+      if (SAMPLE && lane == 0) cta_thr[0] = cta_thr[1] = float_to_ordered(-INFINITY);
     }
     __syncthreads();
     init(acc);
@@ -656,7 +682,7 @@ verify_stream_kernel(const VerifyArgs a) {
         // never fold (and push) at the same time.
         if (__all_sync(__activemask(), bs + kVThreads < vlim)) {
           const int vv[2] = {bs * VEC, (bs + kVThreads) * VEC};
-          fold<T, SAMPLE, 2>(acc, l, m, vv, pr, a.key, a.invT, q, qn, tht, thd);
+          fold<T, SAMPLE, 2>(acc, l, m, vv, pr, a.key, a.invT, q, qn, tht, thd, cta_thr);
           return;
         }
       }
@@ -666,7 +692,7 @@ verify_stream_kernel(const VerifyArgs a) {
         if (idx < vlim) {
           const uint4 l1[1] = {l[k]}, m1[1] = {m[k]};
           const int vv[1] = {idx * VEC};
-          fold<T, SAMPLE, 1>(acc, l1, m1, vv, pr, a.key, a.invT, q, qn, tht, thd);
+          fold<T, SAMPLE, 1>(acc, l1, m1, vv, pr, a.key, a.invT, q, qn, tht, thd, cta_thr);
         }
       }
     };
@@ -689,7 +715,7 @@ verify_stream_kernel(const VerifyArgs a) {
           keep_best(acc.bt, acc.vbt, fmaf(vec_entry<T>(la[0], e), a.invT, g), v + e);
           keep_best(acc.bd, acc.vbd, fmaf(vec_entry<T>(ma[0], e), a.invT, g), v + e);
         }
-        if constexpr (SAMPLE) warp_thresholds(acc, __activemask(), tht, thd);
+        if constexpr (SAMPLE) publish_thresholds(acc, __activemask(), tht, thd, cta_thr);
       }
       fold2(base, la, ma);
       ld2(base + 2 * kStep, la, ma);
