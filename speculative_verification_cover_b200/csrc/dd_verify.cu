@@ -587,6 +587,27 @@ __device__ __forceinline__ uint4 ld_stream(const void* p) {
   return v;
 }
 
+// 16 bytes global -> this thread's own shared-memory slot, asynchronously, caching in
+// L2 only (with a 256-byte L2 prefetch); completion is per thread (commit / wait groups).
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global.L2::256B [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)),
+               "l"(gmem_src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Argmax-only pass (T = 0): each thread stages its own vectors in a ring of
+// kStages half-steps in shared memory, so loads in flight cost no registers and
+// several half-steps are in flight per thread.
+constexpr int kStages = 4;
+constexpr int kRingBytes = kStages * 4 * kVThreads * 16;  // [stage][l0 l1 m0 m1][thread]
+
 template <typename T, bool SAMPLE>
 __global__ void __launch_bounds__(kVThreads, VCfg<SAMPLE>::kMinBlocks)
 verify_stream_kernel(const VerifyArgs a) {
@@ -697,11 +718,38 @@ verify_stream_kernel(const VerifyArgs a) {
       }
     };
     constexpr int kStep = 2 * kVThreads;
+    if constexpr (!SAMPLE) {
+      extern __shared__ uint4 ring[];  // kRingBytes: [stage][4][kVThreads]
+      auto slot = [&](int st, int k) { return ring + (st * 4 + k) * kVThreads + ct; };
+      auto issue = [&](int h) {  // half-step h of this row piece into stage h % kStages
+        const int bs = vbeg + ct + h * kStep, st = h % kStages;
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int idx = bs + k * kVThreads;
+          if (idx < vlim) {
+            cp_async16(slot(st, k), lv + idx);
+            cp_async16(slot(st, 2 + k), mv + idx);
+          }
+        }
+        cp_async_commit();  // a group per half-step, empty or not
+      };
+#pragma unroll
+      for (int h = 0; h < kStages - 1; ++h) issue(h);
+      int h = 0;
+      for (int bs = vbeg + ct; bs < vlim; bs += kStep, ++h) {
+        cp_async_wait<kStages - 2>();  // half-step h has landed (this thread's copies)
+        const int st = h % kStages;
+        const uint4 l[2] = {*slot(st, 0), *slot(st, 1)}, m[2] = {*slot(st, 2), *slot(st, 3)};
+        issue(h + kStages - 1);  // into the stage read one half-step ago
+        fold2(bs, l, m);
+      }
+      cp_async_wait<0>();  // nothing of this row piece left in flight
+    }
     uint4 la[2], ma[2], lb[2], mb[2];
     int base = vbeg + ct;
-    ld2(base, la, ma);
+    if constexpr (SAMPLE) ld2(base, la, ma);
     bool primed = !SAMPLE;
-    for (; base < vlim; base += 2 * kStep) {
+    for (; SAMPLE && base < vlim; base += 2 * kStep) {
       ld2(base + kStep, lb, mb);
       if (!primed) {
         // a first exact score per lane (the four entries of its first vector's first
@@ -875,7 +923,18 @@ cudaError_t launch_verify(const void* lt, const void* lm, int B, int R, int V, i
   a.parts = static_cast<Partial*>(workspace);
   a.maxparts = bound.maxparts > pl.maxparts ? bound.maxparts : pl.maxparts;
   a.spin = spin_limit();
-  verify_stream_kernel<T, SAMPLE><<<pl.grid, kVThreads, 0, stream>>>(a);
+  int smem = 0;
+  if constexpr (!SAMPLE) {
+    smem = kRingBytes;
+    static int configured[64] = {};
+    if (!configured[dev.device & 63]) {
+      cudaError_t e = cudaFuncSetAttribute(verify_stream_kernel<T, SAMPLE>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e != cudaSuccess) return e;
+      configured[dev.device & 63] = 1;
+    }
+  }
+  verify_stream_kernel<T, SAMPLE><<<pl.grid, kVThreads, smem, stream>>>(a);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   verify_merge_kernel<SAMPLE><<<(rows + 7) / 8, 256, 0, stream>>>(a, rows, out);

@@ -104,23 +104,23 @@ class VerifyStep:
         self.select_and_decide()
 
     def forked(self):
-        """The same step with the vocabulary pass on a side stream, concurrent with the
-        attention call (they share no data; selection needs both, so the streams join
-        before it), and the decisions beside the seed selection. The attention kernels
-        leave SMs idle at small shapes and the vocabulary pass fills them."""
+        """The same step on two streams. The vocabulary pass and then the decisions (they
+        read only its statistics) run on a side stream; the attention call runs on the
+        main stream, issued first so that its kernels take SMs ahead of the vocabulary
+        pass. Seed selection needs both, so it waits for the vocabulary pass's event
+        and runs beside the decisions. The attention kernels leave SMs idle at small
+        shapes and the vocabulary pass fills them."""
         main = torch.cuda.current_stream()
         if self.side is None:
             self.side = torch.cuda.Stream(device=main.device)
+            self.verified = torch.cuda.Event()
         self.side.wait_stream(main)
+        self.attention()
         with torch.cuda.stream(self.side):
             self.verify()
-        self.attention()
-        main.wait_stream(self.side)
-        # seed selection (needs both) and the decisions (need only the statistics)
-        # write disjoint outputs: the decisions run beside the selection
-        self.side.wait_stream(main)
-        with torch.cuda.stream(self.side):
+            self.verified.record(self.side)
             self.decide()
+        main.wait_event(self.verified)
         self.select()
         main.wait_stream(self.side)
 
