@@ -52,7 +52,9 @@ typedef enum {
   DD_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misaligned pointer, short workspace */
   DD_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. d = 96) */
   DD_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
-  DD_ERR_TIMEOUT = 4        /* device: a bounded wait ran out (see dd_get_device_error) */
+  DD_ERR_TIMEOUT = 4,       /* device: a bounded wait ran out (see dd_get_device_error) */
+  DD_ERR_BOUNDS = 5         /* device, checked builds only: an index check failed and the
+                               access was skipped (see dd_bounds_checked) */
 } dd_status;
 
 typedef enum { DD_F32 = 0, DD_BF16 = 1 } dd_dtype;
@@ -366,6 +368,34 @@ dd_status dd_selftest_bounded_wait(uint32_t spin_limit, void* stream);
  */
 dd_status dd_selftest_gumbel_screen(float* g_of_level, float* j_of_level, const float* g_req,
                                     float* limit, int n, float* gumbel_max, void* stream);
+
+/*
+ * Checked builds. libdd_checked.so is this library compiled with DD_CHECK_BOUNDS
+ * defined (the Python binding loads it instead of libdd.so when the environment
+ * sets DD_CHECK_BOUNDS=1). In it every index the kernels derive from device data
+ * or from a layout invariant -- a masked row's rank, a partial record's slot, a
+ * seed's rank, the masked-row count, the rows of pass 2's staged inputs -- is
+ * tested before the access. A failed test records DD_ERR_BOUNDS in the device
+ * error word (read by dd_get_device_error; the first error recorded wins), the
+ * access is skipped, and the kernel runs to its end: no trap, no fault, the
+ * context stays usable. Outputs of a call that recorded DD_ERR_BOUNDS are
+ * undefined. Results of calls that record nothing are bit-identical to libdd.so.
+ *
+ * dd_bounds_checked -- 1 in a checked build, 0 otherwise. Pure host function.
+ */
+int dd_bounds_checked(void);
+
+/*
+ * dd_selftest_bounds_check -- self-test of the checked build: one CTA fills a
+ * library-owned device array of 64 ints with 3*i + 1 and reads element `index`
+ * of its first n through the checked path; *value (host pointer) receives the
+ * element, or -1 when the check skipped the read (the device error word then
+ * holds DD_ERR_BOUNDS). Synchronises `stream`.
+ * Errors: DD_ERR_UNSUPPORTED in a build without the checks (nothing is launched,
+ * so no out-of-range read can happen); DD_ERR_INVALID_ARG for value == NULL or n
+ * outside [0, 64].
+ */
+dd_status dd_selftest_bounds_check(int n, int index, int* value, void* stream);
 
 #ifdef __cplusplus
 }

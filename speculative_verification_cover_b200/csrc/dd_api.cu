@@ -232,6 +232,7 @@ const char* dd_status_string(dd_status s) {
     case DD_ERR_UNSUPPORTED: return "DD_ERR_UNSUPPORTED";
     case DD_ERR_CUDA: return "DD_ERR_CUDA";
     case DD_ERR_TIMEOUT: return "DD_ERR_TIMEOUT";
+    case DD_ERR_BOUNDS: return "DD_ERR_BOUNDS";
   }
   return "DD_UNKNOWN_STATUS";
 }
@@ -254,6 +255,20 @@ uint32_t dd_set_spin_limit(uint32_t limit) {
 dd_status dd_selftest_bounded_wait(uint32_t limit, void* stream) {
   if (limit == 0) return DD_ERR_INVALID_ARG;
   return from_cuda(launch_selftest_wait(limit, static_cast<cudaStream_t>(stream)));
+}
+
+int dd_bounds_checked(void) {
+#ifdef DD_CHECK_BOUNDS
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+dd_status dd_selftest_bounds_check(int n, int index, int* value, void* stream) {
+  if (!value || n < 0 || n > 64) return DD_ERR_INVALID_ARG;
+  if (!dd_bounds_checked()) return DD_ERR_UNSUPPORTED;
+  return from_cuda(launch_selftest_bounds(n, index, value, static_cast<cudaStream_t>(stream)));
 }
 
 dd_status dd_selftest_gumbel_screen(float* g_of_level, float* j_of_level, const float* g_req,

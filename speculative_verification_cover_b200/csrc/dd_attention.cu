@@ -116,7 +116,7 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(const PrepArgs a) {
     int before = 0;
     for (int w = 0; w < warp; ++w) before += warp_sums[w];
     const int rank = base + before + incl - 1;
-    if (f) a.mrows[(int64_t)b * L + rank] = i;
+    if (f && DD_IN_BOUNDS(rank >= 0 && rank < L)) a.mrows[(int64_t)b * L + rank] = i;
     if (i < L) a.mrank[(int64_t)b * L + i] = f ? rank : -1;
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -374,7 +374,8 @@ __global__ void __launch_bounds__(128) simt_pass2_kernel(AttnArgs a) {
     const float4 x = Ld<T>::chunk(krow, qd + 4 * e);
     k[e] = make_float4(x.x * sl2, x.y * sl2, x.z * sl2, x.w * sl2);
   }
-  const int nm = a.mcount[b];
+  const int nm0 = a.mcount[b];
+  const int nm = DD_IN_BOUNDS(nm0 >= 0 && nm0 <= L) ? nm0 : 0;
   const int32_t* rows = a.mrows + (int64_t)b * L;
   const float* lse = a.lse + ((int64_t)b * a.Hq + h) * L;
   float acc = 0.f;
@@ -383,11 +384,17 @@ __global__ void __launch_bounds__(128) simt_pass2_kernel(AttnArgs a) {
     for (int t = threadIdx.x; t < QR * (D / 4); t += blockDim.x) {
       const int rr = t / (D / 4), e = t % (D / 4);
       float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (r0 + rr < nm) x = Ld<T>::chunk(qp + (((int64_t)b * L + rows[r0 + rr]) * a.Hq + h) * D, e);
+      if (r0 + rr < nm) {
+        const int row = rows[r0 + rr];
+        if (DD_IN_BOUNDS(row >= 0 && row < L))
+          x = Ld<T>::chunk(qp + (((int64_t)b * L + row) * a.Hq + h) * D, e);
+      }
       Qs[rr][e] = x;
     }
     for (int t = threadIdx.x; t < QR; t += blockDim.x)
-      lse2[t] = (r0 + t < nm) ? lse[rows[r0 + t]] * kLog2e : INFINITY;
+      lse2[t] = (r0 + t < nm && DD_IN_BOUNDS(rows[r0 + t] >= 0 && rows[r0 + t] < L))
+                    ? lse[rows[r0 + t]] * kLog2e
+                    : INFINITY;
     __syncthreads();
     const int nr = min(QR, nm - r0);
     for (int rr = 0; rr < nr; ++rr) {

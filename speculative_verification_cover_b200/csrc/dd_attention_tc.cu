@@ -440,7 +440,7 @@ attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const float lse2 = m + log2f(l);
         p.lse[((int64_t)b * p.Hq + h) * L + i] = lse2 * kLn2;
         if (p.dout_part) p.dout_part[((int64_t)b * p.Hq + h) * L + i] = ln * inv;
-        if (rank >= 0) {
+        if (rank >= 0 && DD_IN_BOUNDS(rank < L)) {
           // pass 2's inputs for a still-masked row: its Q row (from the staged,
           // swizzled tile; q_full completed long before) and its lse in log2 units
           wait_bounded(&bars->q_full, 0, p.spin, abort_flag);
@@ -525,7 +525,9 @@ attn_p2_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
   const int L = p.L;
   const int G = p.Hq / p.Hkv;
   const int col0 = kt * kBN;
-  const int M = p.mcount[b];
+  const int M0 = p.mcount[b];
+  // (the lse window of the last row tile, [m0, m0 + 128), then stays inside Lp)
+  const int M = DD_IN_BOUNDS(M0 >= 0 && M0 <= L) ? M0 : 0;
   const int nrt = (M + 127) / 128;
   const int NT = G * nrt;
   volatile int* abort_flag = &bars->abort_flag;

@@ -470,7 +470,7 @@ attn_p1x2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         const float lse2 = m + log2f(l);
         p.lse[((int64_t)b * p.Hq + h) * L + i] = lse2 * kLn2;
         if (p.dout_part) p.dout_part[((int64_t)b * p.Hq + h) * L + i] = ln * inv;
-        if (rank >= 0) {
+        if (rank >= 0 && DD_IN_BOUNDS(rank < L)) {
           // pass 2's inputs for a still-masked row: its Q row (from the staged,
           // swizzled tile; q_full completed long before) and its lse in log2 units
           wait_bounded(&bars->q_full, 0, p.spin, abort_flag);

@@ -21,6 +21,20 @@ __device__ __forceinline__ void record_error(unsigned int code) {
   atomicCAS(&g_device_error, 0u, code);
 }
 
+// Index checks of the checked build (compiled with DD_CHECK_BOUNDS). Written as
+// `if (DD_IN_BOUNDS(i < n)) access;`: a false condition records DD_ERR_BOUNDS and
+// the access is skipped. Without DD_CHECK_BOUNDS the macro is the constant true
+// and the condition is not evaluated, so normal builds carry no cost.
+#ifdef DD_CHECK_BOUNDS
+__device__ __forceinline__ bool in_bounds_checked(bool ok) {
+  if (!ok) record_error(DD_ERR_BOUNDS);
+  return ok;
+}
+#define DD_IN_BOUNDS(cond) (::dd::in_bounds_checked(cond))
+#else
+#define DD_IN_BOUNDS(cond) true
+#endif
+
 // ---------------------------------------------------------------------------
 // mbarrier helpers (shared::cta). Every wait is bounded by `limit`
 // iterations and by kWaitNs of wall time (a try_wait may suspend the thread

@@ -78,6 +78,7 @@ cudaError_t launch_decide(const dd_decide_params& p, const int32_t* tokens,
                           cudaStream_t stream);
 
 cudaError_t launch_selftest_wait(uint32_t limit, cudaStream_t stream);
+cudaError_t launch_selftest_bounds(int n, int index, int* value, cudaStream_t stream);
 cudaError_t launch_selftest_gumbel(float* g_of_k, float* j_of_k, const float* g_req,
                                    float* limit, int n, cudaStream_t stream);
 float gumbel_max_constant();

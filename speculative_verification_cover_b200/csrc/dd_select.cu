@@ -142,7 +142,8 @@ select_seeds_kernel(const float* __restrict__ entropy, int R, int pos_offset,
                                                                      (tie && before < need)));
       if (sel) {
         const int slot = atomicAdd(&nsel_s, 1);
-        chosen[slot] = ((unsigned long long)key << 32) | (0xFFFFFFFFu - (uint32_t)i);
+        if (DD_IN_BOUNDS(slot < kSelectMaxK))
+          chosen[slot] = ((unsigned long long)key << 32) | (0xFFFFFFFFu - (uint32_t)i);
       }
       if (is_seed) is_seed[(int64_t)b * L + i] = sel ? 1 : 0;
     }
@@ -152,12 +153,13 @@ select_seeds_kernel(const float* __restrict__ entropy, int R, int pos_offset,
     }
   }
   __syncthreads();
-  const int nsel = nsel_s;
+  const int nsel = DD_IN_BOUNDS(nsel_s <= kSelectMaxK && nsel_s <= k) ? nsel_s : 0;
   for (int t = threadIdx.x; t < nsel; t += blockDim.x) {
     const unsigned long long key = chosen[t];
     int rank = 0;
     for (int u = 0; u < nsel; ++u) rank += chosen[u] > key;
-    seeds[(int64_t)b * k + rank] = (int32_t)(0xFFFFFFFFu - (uint32_t)(key & 0xFFFFFFFFull));
+    if (DD_IN_BOUNDS(rank < k))
+      seeds[(int64_t)b * k + rank] = (int32_t)(0xFFFFFFFFu - (uint32_t)(key & 0xFFFFFFFFull));
   }
   for (int t = nsel + threadIdx.x; t < k; t += blockDim.x) seeds[(int64_t)b * k + t] = -1;
   if (count && threadIdx.x == 0) count[b] = nsel;
@@ -247,8 +249,10 @@ decide_kernel(dd_decide_params p, const int32_t* __restrict__ tokens,
     // progress: nothing passed the threshold, so the most confident masked position commits
     const int i = (int)(0xFFFFFFFFu - (uint32_t)(best_key & 0xFFFFFFFFull));
     const int64_t row = (int64_t)b * R + (i - pos_offset);
-    decision[(int64_t)b * L + i] = DD_COMMIT;
-    new_tokens[(int64_t)b * L + i] = sampled ? st.sample_t[row] : st.argmax_t[row];
+    if (DD_IN_BOUNDS(i >= 0 && i < L && i - pos_offset >= 0 && i - pos_offset < R)) {
+      decision[(int64_t)b * L + i] = DD_COMMIT;
+      new_tokens[(int64_t)b * L + i] = sampled ? st.sample_t[row] : st.argmax_t[row];
+    }
   }
 }
 
@@ -294,6 +298,35 @@ cudaError_t launch_decide(const dd_decide_params& p, const int32_t* tokens,
   decide_kernel<<<B, 1024, 0, stream>>>(p, tokens, is_seed, eligible, stats, L, R, pos_offset,
                                        decision, new_tokens, accepted);
   return cudaGetLastError();
+}
+
+// Self-test of the checked build: fill a 64-int array, then read element `index`
+// of its first n through the checked path (-1 when the check skips the read).
+// Without DD_CHECK_BOUNDS the read is not compiled at all.
+__device__ int g_bounds_probe[64];
+__device__ int g_bounds_probe_out;
+__global__ void selftest_bounds_kernel(int n, int index) {
+  for (int t = threadIdx.x; t < 64; t += blockDim.x) g_bounds_probe[t] = 3 * t + 1;
+  __syncthreads();
+  if (threadIdx.x != 0) return;
+  int v = -1;
+#ifdef DD_CHECK_BOUNDS
+  if (DD_IN_BOUNDS(index >= 0 && index < n)) v = g_bounds_probe[index];
+#else
+  (void)n;
+  (void)index;
+#endif
+  g_bounds_probe_out = v;
+}
+
+cudaError_t launch_selftest_bounds(int n, int index, int* value, cudaStream_t stream) {
+  selftest_bounds_kernel<<<1, 64, 0, stream>>>(n, index);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  e = cudaMemcpyFromSymbolAsync(value, g_bounds_probe_out, sizeof(int), 0,
+                                cudaMemcpyDeviceToHost, stream);
+  if (e != cudaSuccess) return e;
+  return cudaStreamSynchronize(stream);
 }
 
 cudaError_t launch_selftest_wait(uint32_t limit, cudaStream_t stream) {

@@ -660,7 +660,7 @@ verify_stream_kernel(const VerifyArgs a) {
       }
       if (lane == 0) {
         const int64_t slot = c - a.split.cta_of(row * spr);
-        a.parts[row * a.maxparts + slot] = r;
+        if (DD_IN_BOUNDS(slot >= 0 && slot < a.maxparts)) a.parts[row * a.maxparts + slot] = r;
       }
       // every warp is past the row: its thresholds start over for the next one
       if (SAMPLE && lane == 0) cta_thr[0] = cta_thr[1] = float_to_ordered(-INFINITY);
@@ -804,7 +804,8 @@ __global__ void __launch_bounds__(256) verify_merge_kernel(const VerifyArgs a, i
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
   const int64_t c0 = a.split.cta_of(row * a.nchunk);
-  const int nparts = (int)(a.split.cta_of(row * a.nchunk + a.nchunk - 1) - c0 + 1);
+  const int np0 = (int)(a.split.cta_of(row * a.nchunk + a.nchunk - 1) - c0 + 1);
+  const int nparts = DD_IN_BOUNDS(np0 >= 1 && np0 <= a.maxparts) ? np0 : 0;
   Partial acc;
   init(acc);
   for (int k = lane; k < nparts; k += 32) merge<SAMPLE>(acc, a.parts[row * a.maxparts + k]);

@@ -4,6 +4,10 @@ Argument marshalling only: sizes are read off the tensors, pointers passed
 as `data_ptr()`, the stream defaults to torch's current CUDA stream. Every
 computation runs in libdd's CUDA kernels; there is no CPU fallback -- CPU
 tensors, a missing library or a non-OK status raise.
+
+With DD_CHECK_BOUNDS=1 in the environment (read when the library is first
+loaded) the binding loads libdd_checked.so, the same library built with device
+index checks (see dd_bounds_checked in include/dd.h).
 """
 from __future__ import annotations
 
@@ -15,8 +19,9 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libdd.so")
+CHECKED_LIB_PATH = os.path.join(_HERE, "libdd_checked.so")
 
-DD_OK, DD_ERR_INVALID_ARG, DD_ERR_UNSUPPORTED, DD_ERR_CUDA, DD_ERR_TIMEOUT = range(5)
+DD_OK, DD_ERR_INVALID_ARG, DD_ERR_UNSUPPORTED, DD_ERR_CUDA, DD_ERR_TIMEOUT, DD_ERR_BOUNDS = range(6)
 DD_F32, DD_BF16 = 0, 1
 POLICIES = {"trust": 0, "kl": 1, "conf": 2, "cover": 3, "coupled": 4, "kl_stochastic": 5}
 DD_NONE, DD_KEEP, DD_REPLACE, DD_REMASK, DD_COMMIT = 0, 1, 2, 3, 4
@@ -29,7 +34,7 @@ EXPORTED = (
     "dd_coupled_gumbel", "dd_select_seeds", "dd_select_seeds_ex", "dd_decide",
     "dd_status_string",
     "dd_get_device_error", "dd_set_spin_limit", "dd_selftest_bounded_wait",
-    "dd_selftest_gumbel_screen",
+    "dd_selftest_gumbel_screen", "dd_bounds_checked", "dd_selftest_bounds_check",
 )
 
 
@@ -55,15 +60,22 @@ class _DecideParams(ctypes.Structure):
 _lib = None
 
 
+def lib_path() -> str:
+    """The library lib() loads: the checked build when DD_CHECK_BOUNDS is set to
+    anything but 0 or the empty string, libdd.so otherwise."""
+    return CHECKED_LIB_PATH if os.environ.get("DD_CHECK_BOUNDS", "0") not in ("", "0") else LIB_PATH
+
+
 def lib():
-    """Load libdd.so (once). Raises ImportError if it has not been built."""
+    """Load the library (once). Raises ImportError if it has not been built."""
     global _lib
     if _lib is not None:
         return _lib
-    if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is missing: build it with "
+    path = lib_path()
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with "
                           "`python -m speculative_verification_cover_b200.build`")
-    L = ctypes.CDLL(LIB_PATH)
+    L = ctypes.CDLL(path)
     P, I, I64, U64, F, SZ = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_uint64,
                              ctypes.c_float, ctypes.c_size_t)
     L.dd_dualview_attention.argtypes = [P] * 8 + [I] * 5 + [F, I, I] + [P] * 5 + [SZ, P]
@@ -99,6 +111,10 @@ def lib():
     L.dd_selftest_bounded_wait.restype = I
     L.dd_selftest_gumbel_screen.argtypes = [P, P, P, P, I, ctypes.POINTER(F), P]
     L.dd_selftest_gumbel_screen.restype = I
+    L.dd_bounds_checked.argtypes = []
+    L.dd_bounds_checked.restype = I
+    L.dd_selftest_bounds_check.argtypes = [I, I, ctypes.POINTER(I), P]
+    L.dd_selftest_bounds_check.restype = I
     _lib = L
     return L
 
@@ -331,3 +347,18 @@ def dd_selftest_gumbel_screen(g_req, stream=None):
         _ptr(g), _ptr(j), _ptr(g_req), _ptr(limit), g_req.numel(), ctypes.byref(gmax),
         _stream(stream)))
     return g, j, limit, float(gmax.value)
+
+
+def dd_bounds_checked() -> bool:
+    """True when the loaded library is the checked build."""
+    return bool(lib().dd_bounds_checked())
+
+
+def dd_selftest_bounds_check(n: int, index: int, stream=None) -> int:
+    """One checked read of element `index` of a 64-int library array (element i
+    holds 3*i + 1) limited to its first n: the value, or -1 when the check skipped
+    the read (dd_get_device_error then returns DD_ERR_BOUNDS)."""
+    v = ctypes.c_int(0)
+    _check("dd_selftest_bounds_check",
+           lib().dd_selftest_bounds_check(int(n), int(index), ctypes.byref(v), _stream(stream)))
+    return int(v.value)

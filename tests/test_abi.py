@@ -185,3 +185,22 @@ def test_select_ex_and_decide_extension_validation(lib):
     p = dd._DecideParams(0, 0.5, 0.9, 0.0, 0.5, 1, 0, 0)
     assert lib.dd_decide(ctypes.byref(p), FAKE, FAKE, FAKE, ctypes.byref(stats), 1, 8, 4, 0,
                          FAKE, FAKE, None, None) == dd.DD_ERR_INVALID_ARG
+
+
+def test_checked_build_exports_the_same_boundary(lib):
+    checked = ctypes.CDLL(build.OUT_CHECKED)
+    for name in declared_symbols():
+        assert hasattr(checked, name), name
+    checked.dd_bounds_checked.restype = ctypes.c_int
+    assert checked.dd_bounds_checked() == 1
+    assert dd.dd_bounds_checked() is False
+
+
+def test_bounds_selftest_refused_without_the_checks(lib):
+    # the normal build launches nothing, so no out-of-range read can happen
+    v = ctypes.c_int(7)
+    assert lib.dd_selftest_bounds_check(64, 100, ctypes.byref(v), None) == dd.DD_ERR_UNSUPPORTED
+    assert v.value == 7
+    assert lib.dd_selftest_bounds_check(65, 0, ctypes.byref(v), None) == dd.DD_ERR_INVALID_ARG
+    assert lib.dd_selftest_bounds_check(64, 0, None, None) == dd.DD_ERR_INVALID_ARG
+    assert lib.dd_status_string(dd.DD_ERR_BOUNDS) == b"DD_ERR_BOUNDS"
