@@ -32,9 +32,15 @@ namespace dd {
 namespace {
 
 constexpr int kVThreads = 256;
+// Launch shape. Each thread stages its own vectors in a shared-memory ring of
+// kStages half-steps (cp.async), so loads in flight cost no registers. The sampling
+// pass needs about 120 registers and runs 2 CTAs per SM (at 3, its registers spill
+// and it is slower).
 template <bool SAMPLE>
 struct VCfg {
   static constexpr int kMinBlocks = SAMPLE ? 2 : 3;  // resident CTAs per SM
+  static constexpr int kStages = 4;
+  static constexpr int kRingBytes = kStages * 4 * kVThreads * 16;  // [stage][l0 l1 m0 m1][thread]
 };
 constexpr int kMaxGridPerSm = 3;
 
@@ -602,16 +608,11 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// Argmax-only pass (T = 0): each thread stages its own vectors in a ring of
-// kStages half-steps in shared memory, so loads in flight cost no registers and
-// several half-steps are in flight per thread.
-constexpr int kStages = 4;
-constexpr int kRingBytes = kStages * 4 * kVThreads * 16;  // [stage][l0 l1 m0 m1][thread]
-
 template <typename T, bool SAMPLE>
 __global__ void __launch_bounds__(kVThreads, VCfg<SAMPLE>::kMinBlocks)
 verify_stream_kernel(const VerifyArgs a) {
   constexpr int VEC = Vec<T>::N;
+  constexpr int kStages = VCfg<SAMPLE>::kStages;
   __shared__ Partial red[kVThreads / 32];
 
   const int c = blockIdx.x;
@@ -679,18 +680,6 @@ verify_stream_kernel(const VerifyArgs a) {
     const uint4* lv = reinterpret_cast<const uint4*>(LT + row * a.ld);
     const uint4* mv = reinterpret_cast<const uint4*>(LM + row * a.ld);
     const int vlim = min(vend, nvr);  // slots past nvr carry no full vector
-    // Two vectors per matrix per half-step; while one pair is folded the next
-    // pair's loads are in flight (ping-pong, no register moves).
-    auto ld2 = [&](int bs, uint4 (&l)[2], uint4 (&m)[2]) {
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        const int idx = bs + k * kVThreads;
-        if (idx < vlim) {
-          l[k] = ld_stream(lv + idx);
-          m[k] = ld_stream(mv + idx);
-        }
-      }
-    };
     // per-row parts of the noise generator (only used when sampling)
     const PhiloxRow pr = philox_row((uint32_t)pos, (uint32_t)b, a.key.step, a.key.k0, a.key.k1);
     float tht = -INFINITY, thd = -INFINITY;  // the screen's thresholds (warp-uniform)
@@ -718,7 +707,7 @@ verify_stream_kernel(const VerifyArgs a) {
       }
     };
     constexpr int kStep = 2 * kVThreads;
-    if constexpr (!SAMPLE) {
+    {
       extern __shared__ uint4 ring[];  // kRingBytes: [stage][4][kVThreads]
       auto slot = [&](int st, int k) { return ring + (st * 4 + k) * kVThreads + ct; };
       auto issue = [&](int h) {  // half-step h of this row piece into stage h % kStages
@@ -741,33 +730,24 @@ verify_stream_kernel(const VerifyArgs a) {
         const int st = h % kStages;
         const uint4 l[2] = {*slot(st, 0), *slot(st, 1)}, m[2] = {*slot(st, 2), *slot(st, 3)};
         issue(h + kStages - 1);  // into the stage read one half-step ago
+        if constexpr (SAMPLE) {
+          if (h == 0) {
+            // a first exact score per lane (the four entries of its first vector's first
+            // generator counter), so the screen has a threshold from the start
+            const int v = bs * VEC;
+            const PhiloxOut o = philox_row_counter(pr, (uint32_t)(v >> 2), a.key.k0, a.key.k1);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float g = gumbel_from_word(o.w[e]);
+              keep_best(acc.bt, acc.vbt, fmaf(vec_entry<T>(l[0], e), a.invT, g), v + e);
+              keep_best(acc.bd, acc.vbd, fmaf(vec_entry<T>(m[0], e), a.invT, g), v + e);
+            }
+            publish_thresholds(acc, __activemask(), tht, thd, cta_thr);
+          }
+        }
         fold2(bs, l, m);
       }
       cp_async_wait<0>();  // nothing of this row piece left in flight
-    }
-    uint4 la[2], ma[2], lb[2], mb[2];
-    int base = vbeg + ct;
-    if constexpr (SAMPLE) ld2(base, la, ma);
-    bool primed = !SAMPLE;
-    for (; SAMPLE && base < vlim; base += 2 * kStep) {
-      ld2(base + kStep, lb, mb);
-      if (!primed) {
-        // a first exact score per lane (the four entries of its first vector's first
-        // generator counter), so the screen has a threshold from the start
-        primed = true;
-        const int v = base * VEC;
-        const PhiloxOut o = philox_row_counter(pr, (uint32_t)(v >> 2), a.key.k0, a.key.k1);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float g = gumbel_from_word(o.w[e]);
-          keep_best(acc.bt, acc.vbt, fmaf(vec_entry<T>(la[0], e), a.invT, g), v + e);
-          keep_best(acc.bd, acc.vbd, fmaf(vec_entry<T>(ma[0], e), a.invT, g), v + e);
-        }
-        if constexpr (SAMPLE) publish_thresholds(acc, __activemask(), tht, thd, cta_thr);
-      }
-      fold2(base, la, ma);
-      ld2(base + 2 * kStep, la, ma);
-      fold2(base + kStep, lb, mb);
     }
     if (vend == spr) {
       // ragged end of the row (fewer than 16 bytes): one entry per thread
@@ -924,9 +904,8 @@ cudaError_t launch_verify(const void* lt, const void* lm, int B, int R, int V, i
   a.parts = static_cast<Partial*>(workspace);
   a.maxparts = bound.maxparts > pl.maxparts ? bound.maxparts : pl.maxparts;
   a.spin = spin_limit();
-  int smem = 0;
-  if constexpr (!SAMPLE) {
-    smem = kRingBytes;
+  const int smem = VCfg<SAMPLE>::kRingBytes;
+  {
     static int configured[64] = {};
     if (!configured[dev.device & 63]) {
       cudaError_t e = cudaFuncSetAttribute(verify_stream_kernel<T, SAMPLE>,
