@@ -15,9 +15,11 @@
 // (rows x vectors per row); it is split into equal contiguous ranges, one per
 // persistent CTA (several per SM), so every SM streams the same number of bytes
 // whatever B, R and V are. A CTA's range is one to a few row pieces; in each
-// piece its 256 threads stride over the vectors four at a time with streaming
-// 16-byte loads, folding each into an online (running-max rescaled) state kept
-// in float2 lanes so pairs of entries use the packed fp32 pipe:
+// piece its 256 threads stride over the vectors, two per matrix per half-step,
+// each thread staging its own 16-byte vectors through a ring of four half-steps
+// in shared memory (cp.async), and fold each into an online (running-max
+// rescaled) state kept in float2 lanes so pairs of entries use the packed fp32
+// pipe:
 //   s1 = sum e^{x - M},  s2 = sum e^{x - M} (x - M) log2(e),  sk = sum e^{m - Md}(m - l).
 // At the end of a piece the CTA reduces its state to one partial per
 // (row, CTA) in the workspace; a small second kernel merges a row's partials:
@@ -584,14 +586,6 @@ struct VerifyArgs {
   int maxparts;
   uint32_t spin;
 };
-
-__device__ __forceinline__ uint4 ld_stream(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
 
 // 16 bytes global -> this thread's own shared-memory slot, asynchronously, caching in
 // L2 only (with a 256-byte L2 prefetch); completion is per thread (commit / wait groups).

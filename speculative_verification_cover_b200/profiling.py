@@ -7,8 +7,9 @@ RAW_CSV is the output of `ncu -i <report> --page raw --csv` (one row per capture
 launch). The record for KERNEL -- dram__bytes_read.sum + dram__bytes_write.sum per
 launch, averaged over the captured launches of that kernel -- is written to
 profiles/traffic.json together with the workload, the command and a hash of the
-kernel's source file, so that a reader (bench.py) can tell whether the figure
-still describes the current kernel. Nothing here is edited by hand.
+kernel's source code (comments and layout ignored), so that a reader (bench.py)
+can tell whether the figure still describes the current kernel. Nothing here is
+edited by hand.
 """
 from __future__ import annotations
 
@@ -17,6 +18,7 @@ import csv
 import hashlib
 import json
 import os
+import re
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
@@ -26,9 +28,18 @@ _UNITS = {"byte": 1.0, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "Tbyte": 1e12,
           "KB": 1e3, "MB": 1e6, "GB": 1e9}
 
 
+def _code_only(text: str) -> str:
+    """The source with comments removed and whitespace runs collapsed: what the
+    compiler sees, so that an edit to a comment does not retire a measurement."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def source_hash(path: str) -> str:
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    """Hash of a kernel source's code (comments and layout ignored)."""
+    with open(path, encoding="utf-8") as f:
+        return hashlib.sha256(_code_only(f.read()).encode()).hexdigest()[:16]
 
 
 def dram_bytes_per_launch(raw_csv: str, kernel: str):

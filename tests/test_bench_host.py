@@ -41,7 +41,7 @@ def test_traffic_record_parses_ncu_raw_csv_and_goes_stale(tmp_path):
     assert n == 2
     assert per == pytest.approx((200.5e6 + 3.45e6 + 199.5e6 + 3.55e6) / 2)
     src = tmp_path / "k.cu"
-    src.write_text("// kernel v1\n")
+    src.write_text("// kernel v1\nint a = 1;\n")
     out = tmp_path / "traffic.json"
     rec = profiling.record(str(raw), "verify_stream_kernel", "wl", str(src), "ncu ...",
                            out=str(out))
@@ -53,7 +53,10 @@ def test_traffic_record_parses_ncu_raw_csv_and_goes_stale(tmp_path):
     out.write_text(json.dumps(db))
     assert profiling.lookup("verify_stream_kernel", "wl", path=str(out)) == pytest.approx(per)
     assert profiling.lookup("verify_stream_kernel", "other", path=str(out)) is None
-    src.write_text("// kernel v2\n")  # the kernel changed since the capture
+    # comments and layout are not the kernel: the record still holds
+    src.write_text("/* the same kernel,\n   re-commented */ int  a =\n 1; // v1.1\n")
+    assert profiling.lookup("verify_stream_kernel", "wl", path=str(out)) == pytest.approx(per)
+    src.write_text("// kernel v2\nint a = 2;\n")  # the kernel changed since the capture
     assert profiling.lookup("verify_stream_kernel", "wl", path=str(out)) is None
     with pytest.raises(ValueError):
         profiling.dram_bytes_per_launch(str(raw), "no_such_kernel")
