@@ -141,6 +141,7 @@ struct HeadReduce {
 };
 __global__ void __launch_bounds__(256) head_reduce_kernel(HeadReduce r0, HeadReduce r1, int B, int L,
                                                           float inv_hq, int accumulate) {
+  pdl_wait();  // launched as a dependent of the previous kernel
   const int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   const int64_t pos = t >> 3;
   const int sub = (int)(t & 7);
@@ -485,8 +486,9 @@ cudaError_t launch_attention(const AttnArgs& a, cudaStream_t stream) {
     else if (!a.accumulate) cudaMemsetAsync(a.d_in, 0, total * sizeof(float), stream);
   }
   if (rin.part || rout.part) {
-    head_reduce_kernel<<<(unsigned)((total * 8 + 255) / 256), 256, 0, stream>>>(
-        rin, rout, a.B, a.L, a.stats_weight / a.Hq, a.accumulate);
+    err = launch_dependent(head_reduce_kernel, dim3((unsigned)((total * 8 + 255) / 256)), dim3(256),
+                           0, stream, rin, rout, a.B, a.L, a.stats_weight / a.Hq, a.accumulate);
+    if (err != cudaSuccess) return err;
   }
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   return cudaSuccess;

@@ -147,6 +147,9 @@ attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   __syncthreads();
   fence_after_sync();
   const uint32_t tmem = bars->tmem_base;
+  // set-up above touches only shared and tensor memory; the previous kernel's
+  // outputs are read from here on
+  pdl_wait();
 
   if (warp == 0) {
     // ------------------------------------------------------------------ producer
@@ -525,11 +528,6 @@ attn_p2_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
   const int L = p.L;
   const int G = p.Hq / p.Hkv;
   const int col0 = kt * kBN;
-  const int M0 = p.mcount[b];
-  // (the lse window of the last row tile, [m0, m0 + 128), then stays inside Lp)
-  const int M = DD_IN_BOUNDS(M0 >= 0 && M0 <= L) ? M0 : 0;
-  const int nrt = (M + 127) / 128;
-  const int NT = G * nrt;
   volatile int* abort_flag = &bars->abort_flag;
 
   if (threadIdx.x == 0) {
@@ -551,6 +549,14 @@ attn_p2_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
   __syncthreads();
   fence_after_sync();
   const uint32_t tmem = bars->tmem_base;
+  // set-up above touches only shared and tensor memory; the previous kernel's
+  // outputs (the masked-row count, Q_m, lse) are read from here on
+  pdl_wait();
+  const int M0 = p.mcount[b];
+  // (the lse window of the last row tile, [m0, m0 + 128), then stays inside Lp)
+  const int M = DD_IN_BOUNDS(M0 >= 0 && M0 <= L) ? M0 : 0;
+  const int nrt = (M + 127) / 128;
+  const int NT = G * nrt;
 
   if (warp == 0) {
     // ------------------------------------------------------------------ producer
@@ -754,8 +760,7 @@ cudaError_t launch_p1(const AttnArgs& a, bool pass2, cudaStream_t stream) {
     configured[di.device & 63] = 1;
   }
   dim3 grid((a.L - a.q_begin + kBM - 1) / kBM, a.Hq, a.B);
-  attn_p1_kernel<D><<<grid, kP1Threads, smem, stream>>>(tq, tk, tv, p);
-  return cudaGetLastError();
+  return launch_dependent(attn_p1_kernel<D>, grid, dim3(kP1Threads), smem, stream, tq, tk, tv, p);
 }
 
 template <int D>
@@ -784,8 +789,7 @@ cudaError_t launch_p2(const AttnArgs& a, cudaStream_t stream) {
   p.din_part = a.din_part;
   p.spin = spin_limit();
   dim3 grid((a.L + kBN - 1) / kBN, a.Hkv, a.B);
-  attn_p2_kernel<D><<<grid, kP2Threads, smem, stream>>>(tk, tqm, p);
-  return cudaGetLastError();
+  return launch_dependent(attn_p2_kernel<D>, grid, dim3(kP2Threads), smem, stream, tk, tqm, p);
 }
 
 }  // namespace

@@ -156,6 +156,9 @@ attn_p1x2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   __syncthreads();
   fence_after_sync();
   const uint32_t tmem = bars->tmem_base;
+  // set-up above touches only shared and tensor memory; the previous kernel's
+  // outputs are read from here on
+  pdl_wait();
 
   if (warp == 0) {
     // ------------------------------------------------------------------ producer
@@ -520,8 +523,8 @@ cudaError_t launch_p1x2(const AttnArgs& a, bool pass2, cudaStream_t stream) {
     configured[dev & 63] = 1;
   }
   dim3 grid((a.L - a.q_begin + 2 * kBM - 1) / (2 * kBM), a.Hq, a.B);
-  attn_p1x2_kernel<D><<<grid, kP1x2Threads, smem, stream>>>(tq, tk, tv, p);
-  return cudaGetLastError();
+  return launch_dependent(attn_p1x2_kernel<D>, grid, dim3(kP1x2Threads), smem, stream, tq, tk, tv,
+                          p);
 }
 
 template cudaError_t launch_p1x2<64>(const AttnArgs&, bool, cudaStream_t);

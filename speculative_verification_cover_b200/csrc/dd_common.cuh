@@ -21,6 +21,13 @@ __device__ __forceinline__ void record_error(unsigned int code) {
   atomicCAS(&g_device_error, 0u, code);
 }
 
+// Programmatic dependent launch. A kernel launched by launch_dependent() may be
+// scheduled while the previous kernel on its stream is still finishing (once every
+// CTA of that kernel has started); it calls pdl_wait() before it reads anything that
+// kernel writes, or writes anything it reads. Without the launch attribute the wait
+// returns at once.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Index checks of the checked build (compiled with DD_CHECK_BOUNDS). Written as
 // `if (DD_IN_BOUNDS(i < n)) access;`: a false condition records DD_ERR_BOUNDS and
 // the access is skipped. Without DD_CHECK_BOUNDS the macro is the constant true

@@ -57,6 +57,25 @@ AttnWorkspace attn_workspace_layout(int B, int L, int Hq, int Hkv, int d);
 
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t stream);
 
+// Launch `kernel` so that it may start while the previous kernel on `stream` is still
+// finishing (programmatic stream serialization); the kernel calls pdl_wait() before
+// it touches that kernel's data.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                             cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 cudaError_t launch_verify_logits(const void* lt, const void* lm, dd_dtype dtype, int B, int R,
                                  int V, int64_t ld, int pos_offset, float temperature,
                                  uint64_t seed, uint64_t step, const dd_row_stats& out,

@@ -55,6 +55,7 @@ select_seeds_kernel(const float* __restrict__ entropy, int R, int pos_offset,
                     const uint8_t* __restrict__ eligible, int L, int k, float min_score,
                     int32_t* __restrict__ seeds, uint8_t* __restrict__ is_seed,
                     float* __restrict__ score, int32_t* __restrict__ count) {
+  pdl_wait();  // launched as a dependent of the previous kernel
   extern __shared__ uint32_t skey[];  // [L] orderable score; 0 = not a candidate
   __shared__ unsigned int hist[256];
   __shared__ int warp_tmp[32];
@@ -174,6 +175,7 @@ decide_kernel(dd_decide_params p, const int32_t* __restrict__ tokens,
               const uint8_t* __restrict__ is_seed, const uint8_t* __restrict__ eligible,
               dd_row_stats st, int L, int R, int pos_offset, uint8_t* __restrict__ decision,
               int32_t* __restrict__ new_tokens, uint8_t* __restrict__ accepted) {
+  pdl_wait();  // launched as a dependent of the previous kernel
   const int b = blockIdx.x;
   const bool sampled = p.temperature > 0.f;
   const bool commit_on = p.tau_commit > 0.f;
@@ -284,10 +286,9 @@ cudaError_t launch_select_seeds(const float* entropy, int R, int pos_offset, con
     if (e != cudaSuccess) return e;
     configured_for = dev.device;
   }
-  select_seeds_kernel<<<B, kSelThreads, smem, stream>>>(entropy, R, pos_offset, d_in, d_out,
-                                                        eligible, L, k, min_score, seeds, is_seed,
-                                                        score, count);
-  return cudaGetLastError();
+  return launch_dependent(select_seeds_kernel, dim3(B), dim3(kSelThreads), smem, stream, entropy, R,
+                          pos_offset, d_in, d_out, eligible, L, k, min_score, seeds, is_seed,
+                          score, count);
 }
 
 cudaError_t launch_decide(const dd_decide_params& p, const int32_t* tokens,
@@ -295,9 +296,8 @@ cudaError_t launch_decide(const dd_decide_params& p, const int32_t* tokens,
                           const dd_row_stats& stats, int B, int L, int R, int pos_offset,
                           uint8_t* decision, int32_t* new_tokens, uint8_t* accepted,
                           cudaStream_t stream) {
-  decide_kernel<<<B, 1024, 0, stream>>>(p, tokens, is_seed, eligible, stats, L, R, pos_offset,
-                                       decision, new_tokens, accepted);
-  return cudaGetLastError();
+  return launch_dependent(decide_kernel, dim3(B), dim3(1024), 0, stream, p, tokens, is_seed, eligible,
+                          stats, L, R, pos_offset, decision, new_tokens, accepted);
 }
 
 // Self-test of the checked build: fill a 64-int array, then read element `index`

@@ -774,6 +774,7 @@ verify_stream_kernel(const VerifyArgs a) {
 template <bool SAMPLE>
 __global__ void __launch_bounds__(256) verify_merge_kernel(const VerifyArgs a, int rows,
                                                            dd_row_stats out) {
+  pdl_wait();  // launched as a dependent of the previous kernel
   const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
@@ -911,8 +912,8 @@ cudaError_t launch_verify(const void* lt, const void* lm, int B, int R, int V, i
   verify_stream_kernel<T, SAMPLE><<<pl.grid, kVThreads, smem, stream>>>(a);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  verify_merge_kernel<SAMPLE><<<(rows + 7) / 8, 256, 0, stream>>>(a, rows, out);
-  return cudaGetLastError();
+  return launch_dependent(verify_merge_kernel<SAMPLE>, dim3((rows + 7) / 8), dim3(256), 0, stream, a,
+                          rows, out);
 }
 
 }  // namespace
