@@ -680,15 +680,16 @@ verify_stream_kernel(const VerifyArgs a) {
     // both vectors of a half-step in one fold where both exist (one warp-wide
     // screening threshold per pair), else the one that does
     auto fold2 = [&](int bs, const uint4 (&l)[2], const uint4 (&m)[2]) {
-      if constexpr (SAMPLE) {
-        // The two-vector fold only when every active lane of the warp has both: the
-        // warp's lanes share one queue and one count, so two groups of a warp must
-        // never fold (and push) at the same time.
-        if (__all_sync(__activemask(), bs + kVThreads < vlim)) {
-          const int vv[2] = {bs * VEC, (bs + kVThreads) * VEC};
-          fold<T, SAMPLE, 2>(acc, l, m, vv, pr, a.key, a.invT, q, qn, tht, thd, cta_thr);
-          return;
-        }
+      // Both vectors in one fold (one maximum update and rescale check for the pair)
+      // where both exist. When sampling, only if every active lane of the warp has
+      // both: the warp's lanes share one queue and one count, so two groups of a warp
+      // must never fold (and push) at the same time.
+      const bool both = SAMPLE ? __all_sync(__activemask(), bs + kVThreads < vlim)
+                               : bs + kVThreads < vlim;
+      if (both) {
+        const int vv[2] = {bs * VEC, (bs + kVThreads) * VEC};
+        fold<T, SAMPLE, 2>(acc, l, m, vv, pr, a.key, a.invT, q, qn, tht, thd, cta_thr);
+        return;
       }
 #pragma unroll
       for (int k = 0; k < 2; ++k) {
