@@ -704,27 +704,34 @@ verify_stream_kernel(const VerifyArgs a) {
     constexpr int kStep = 2 * kVThreads;
     {
       extern __shared__ uint4 ring[];  // kRingBytes: [stage][4][kVThreads]
-      auto slot = [&](int st, int k) { return ring + (st * 4 + k) * kVThreads + ct; };
-      auto issue = [&](int h) {  // half-step h of this row piece into stage h % kStages
-        const int bs = vbeg + ct + h * kStep, st = h % kStages;
+      static_assert((kStages & (kStages - 1)) == 0, "stages: a power of two");
+      constexpr int kStageStride = 4 * kVThreads;  // uint4s per stage
+      uint4* const mine = ring + ct;               // this thread's slot 0 of stage 0
+      // the issue cursor: next half-step's stage and the index of its first vector
+      int ist = 0, ibs = vbeg + ct;
+      auto issue = [&]() {
+        uint4* const sp = mine + ist * kStageStride;
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
-          const int idx = bs + k * kVThreads;
+          const int idx = ibs + k * kVThreads;
           if (idx < vlim) {
-            cp_async16(slot(st, k), lv + idx);
-            cp_async16(slot(st, 2 + k), mv + idx);
+            cp_async16(sp + k * kVThreads, lv + idx);
+            cp_async16(sp + (2 + k) * kVThreads, mv + idx);
           }
         }
         cp_async_commit();  // a group per half-step, empty or not
+        ist = (ist + 1) & (kStages - 1);
+        ibs += kStep;
       };
 #pragma unroll
-      for (int h = 0; h < kStages - 1; ++h) issue(h);
-      int h = 0;
+      for (int hh = 0; hh < kStages - 1; ++hh) issue();
+      int h = 0, cst = 0;
       for (int bs = vbeg + ct; bs < vlim; bs += kStep, ++h) {
         cp_async_wait<kStages - 2>();  // half-step h has landed (this thread's copies)
-        const int st = h % kStages;
-        const uint4 l[2] = {*slot(st, 0), *slot(st, 1)}, m[2] = {*slot(st, 2), *slot(st, 3)};
-        issue(h + kStages - 1);  // into the stage read one half-step ago
+        const uint4* const sp = mine + cst * kStageStride;
+        const uint4 l[2] = {sp[0], sp[kVThreads]}, m[2] = {sp[2 * kVThreads], sp[3 * kVThreads]};
+        cst = (cst + 1) & (kStages - 1);
+        issue();  // into the stage read one half-step ago
         if constexpr (SAMPLE) {
           if (h == 0) {
             // a first exact score per lane (the four entries of its first vector's first
