@@ -15,8 +15,8 @@
 // (rows x vectors per row); it is split into equal contiguous ranges, one per
 // persistent CTA (several per SM), so every SM streams the same number of bytes
 // whatever B, R and V are. A CTA's range is one to a few row pieces; in each
-// piece its 256 threads stride over the vectors, two per matrix per half-step,
-// each thread staging its own 16-byte vectors through a ring of four half-steps
+// piece its 128 threads stride over the vectors, two per matrix per half-step,
+// each thread staging its own 16-byte vectors through a ring of three half-steps
 // in shared memory (cp.async), and fold each into an online (running-max
 // rescaled) state kept in float2 lanes so pairs of entries use the packed fp32
 // pipe:
@@ -33,18 +33,20 @@ namespace dd {
 
 namespace {
 
-constexpr int kVThreads = 256;
+constexpr int kVThreads = 128;
 // Launch shape. Each thread stages its own vectors in a shared-memory ring of
-// kStages half-steps (cp.async), so loads in flight cost no registers. The sampling
-// pass needs about 120 registers and runs 2 CTAs per SM (at 3, its registers spill
-// and it is slower).
+// kStages half-steps (cp.async), so loads in flight cost no registers. CTAs are
+// small -- 128 threads, about 10 K registers and 24 KB of shared memory at T = 0 --
+// so that one fits on an SM beside a CTA of the attention's pass 1 (the two calls of a
+// verification step run side by side) and the SM's several CTAs share its bandwidth
+// in fine steps. The sampling pass needs about 120 registers: 4 CTAs per SM.
 template <bool SAMPLE>
 struct VCfg {
-  static constexpr int kMinBlocks = SAMPLE ? 2 : 3;  // resident CTAs per SM
-  static constexpr int kStages = 4;
+  static constexpr int kMinBlocks = SAMPLE ? 4 : 6;  // resident CTAs per SM
+  static constexpr int kStages = 3;
   static constexpr int kRingBytes = kStages * 4 * kVThreads * 16;  // [stage][l0 l1 m0 m1][thread]
 };
-constexpr int kMaxGridPerSm = 3;
+constexpr int kMaxGridPerSm = 6;  // bounds the grid for workspace sizing
 
 struct Partial {
   float mt, s1t, s2t;  // verifier: max, sum e, sum e*y (log2 units)
@@ -704,7 +706,6 @@ verify_stream_kernel(const VerifyArgs a) {
     constexpr int kStep = 2 * kVThreads;
     {
       extern __shared__ uint4 ring[];  // kRingBytes: [stage][4][kVThreads]
-      static_assert((kStages & (kStages - 1)) == 0, "stages: a power of two");
       constexpr int kStageStride = 4 * kVThreads;  // uint4s per stage
       uint4* const mine = ring + ct;               // this thread's slot 0 of stage 0
       // the issue cursor: next half-step's stage and the index of its first vector
@@ -720,7 +721,7 @@ verify_stream_kernel(const VerifyArgs a) {
           }
         }
         cp_async_commit();  // a group per half-step, empty or not
-        ist = (ist + 1) & (kStages - 1);
+        ist = ist + 1 == kStages ? 0 : ist + 1;
         ibs += kStep;
       };
 #pragma unroll
@@ -730,7 +731,7 @@ verify_stream_kernel(const VerifyArgs a) {
         cp_async_wait<kStages - 2>();  // half-step h has landed (this thread's copies)
         const uint4* const sp = mine + cst * kStageStride;
         const uint4 l[2] = {sp[0], sp[kVThreads]}, m[2] = {sp[2 * kVThreads], sp[3 * kVThreads]};
-        cst = (cst + 1) & (kStages - 1);
+        cst = cst + 1 == kStages ? 0 : cst + 1;
         issue();  // into the stage read one half-step ago
         if constexpr (SAMPLE) {
           if (h == 0) {
