@@ -149,6 +149,28 @@ dd_status dd_dualview_attention_ex(
     void* out, float* lse, float* d_in, float* d_out,
     void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * dd_dualview_attention_ex2 -- dd_dualview_attention_ex that also records
+ * `prep_done` (a cudaEvent_t created by the caller; NULL: none) on `stream` right
+ * after the call's first kernel, the mask preparation. That kernel lets the first
+ * attention pass take its SMs while it runs, so by the time the event completes
+ * the pass is resident. A caller that runs a bandwidth-bound kernel beside this
+ * call on another stream (the vocabulary pass of the same verification step) makes
+ * that stream wait on the event: the other kernel then fills the SMs the pass
+ * leaves free instead of taking every SM before the pass can start. The event
+ * says nothing about the call's outputs; wait for the call itself before reading
+ * them. Every other argument, and the errors, as dd_dualview_attention_ex (plus
+ * DD_ERR_CUDA if the event cannot be recorded).
+ */
+dd_status dd_dualview_attention_ex2(
+    const void* q, const void* k_cur, const void* v_cur,
+    const void* k_prev, const void* v_prev,
+    const uint8_t* is_seed, const uint8_t* is_masked, const uint8_t* is_new,
+    int B, int L, int Hq, int Hkv, int d, float softmax_scale, dd_dtype dtype,
+    int q_begin, int accumulate_stats, float stats_weight,
+    void* out, float* lse, float* d_in, float* d_out,
+    void* workspace, size_t workspace_bytes, void* prep_done, void* stream);
+
 /* Bytes of device scratch dd_dualview_attention needs for these sizes
  * (0 on invalid sizes). Pure host function. Dominant terms: a bf16 copy of K
  * and V with the seed rows taken from the cache (2*B*L*Hkv*d*2 bytes) and room

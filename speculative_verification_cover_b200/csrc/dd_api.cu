@@ -68,13 +68,14 @@ size_t dd_dualview_attention_workspace_size(int B, int L, int Hq, int Hkv, int d
   return attn_workspace_layout(B, L, Hq, Hkv, d).total;
 }
 
-dd_status dd_dualview_attention_ex(const void* q, const void* k_cur, const void* v_cur,
-                                   const void* k_prev, const void* v_prev, const uint8_t* is_seed,
-                                   const uint8_t* is_masked, const uint8_t* is_new, int B, int L,
-                                   int Hq, int Hkv, int d, float softmax_scale, dd_dtype dtype,
-                                   int q_begin, int accumulate_stats, float stats_weight,
-                                   void* out, float* lse, float* d_in, float* d_out,
-                                   void* workspace, size_t workspace_bytes, void* stream) {
+dd_status dd_dualview_attention_ex2(const void* q, const void* k_cur, const void* v_cur,
+                                    const void* k_prev, const void* v_prev, const uint8_t* is_seed,
+                                    const uint8_t* is_masked, const uint8_t* is_new, int B, int L,
+                                    int Hq, int Hkv, int d, float softmax_scale, dd_dtype dtype,
+                                    int q_begin, int accumulate_stats, float stats_weight,
+                                    void* out, float* lse, float* d_in, float* d_out,
+                                    void* workspace, size_t workspace_bytes, void* prep_done,
+                                    void* stream) {
   if (!q || !k_cur || !v_cur || !out || !lse) return DD_ERR_INVALID_ARG;
   if (q_begin < 0 || q_begin >= L) return DD_ERR_INVALID_ARG;
   if (!(stats_weight == stats_weight) || isinf(stats_weight)) return DD_ERR_INVALID_ARG;
@@ -113,7 +114,21 @@ dd_status dd_dualview_attention_ex(const void* q, const void* k_cur, const void*
   a.q_m = w + ws.qm_off;
   a.lse2_m = reinterpret_cast<float*>(w + ws.lse2m_off);
   a.Lp = ws.Lp;
-  return from_cuda(launch_attention(a, static_cast<cudaStream_t>(stream)));
+  return from_cuda(launch_attention(a, static_cast<cudaStream_t>(stream),
+                                    static_cast<cudaEvent_t>(prep_done)));
+}
+
+dd_status dd_dualview_attention_ex(const void* q, const void* k_cur, const void* v_cur,
+                                   const void* k_prev, const void* v_prev, const uint8_t* is_seed,
+                                   const uint8_t* is_masked, const uint8_t* is_new, int B, int L,
+                                   int Hq, int Hkv, int d, float softmax_scale, dd_dtype dtype,
+                                   int q_begin, int accumulate_stats, float stats_weight,
+                                   void* out, float* lse, float* d_in, float* d_out,
+                                   void* workspace, size_t workspace_bytes, void* stream) {
+  return dd_dualview_attention_ex2(q, k_cur, v_cur, k_prev, v_prev, is_seed, is_masked, is_new,
+                                   B, L, Hq, Hkv, d, softmax_scale, dtype, q_begin,
+                                   accumulate_stats, stats_weight, out, lse, d_in, d_out,
+                                   workspace, workspace_bytes, nullptr, stream);
 }
 
 dd_status dd_dualview_attention(const void* q, const void* k_cur, const void* v_cur,

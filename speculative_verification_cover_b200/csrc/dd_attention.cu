@@ -63,6 +63,9 @@ constexpr int kPrepThreads = 1024;
 constexpr int kPrepUnitsPerThread = 4;
 
 __global__ void __launch_bounds__(kPrepThreads) prep_kernel(const PrepArgs a) {
+  // Pass 1 may take its SMs (and set up its barriers and tensor memory) while this
+  // kernel runs; it reads nothing of ours before its pdl_wait().
+  pdl_release();
   const int b = blockIdx.y;
   const int L = a.L;
   if (blockIdx.x > 0) {
@@ -433,7 +436,7 @@ cudaError_t launch_simt(const AttnArgs& a, cudaStream_t stream) {
 cudaError_t launch_attention_tc(const AttnArgs& a, cudaStream_t stream, bool* handled,
                                 int* din_slices);
 
-cudaError_t launch_attention(const AttnArgs& a, cudaStream_t stream) {
+cudaError_t launch_attention(const AttnArgs& a, cudaStream_t stream, cudaEvent_t prep_done) {
   cudaError_t err;
   const bool need_din = a.d_in != nullptr && a.is_masked != nullptr;
   PrepArgs pa{};
@@ -461,6 +464,7 @@ cudaError_t launch_attention(const AttnArgs& a, cudaStream_t stream) {
   }
   prep_kernel<<<dim3(1 + copy_blocks, a.B), kPrepThreads, 0, stream>>>(pa);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  if (prep_done != nullptr && (err = cudaEventRecord(prep_done, stream)) != cudaSuccess) return err;
   bool handled = false;
   int din_slices = a.Hq;  // d_in partials: per query head (CUDA-core pass 2) or per kv head
   if (a.dtype == DD_BF16) {

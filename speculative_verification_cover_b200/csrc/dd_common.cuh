@@ -27,6 +27,9 @@ __device__ __forceinline__ void record_error(unsigned int code) {
 // kernel writes, or writes anything it reads. Without the launch attribute the wait
 // returns at once.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Let the next kernel on the stream (launched with launch_dependent) be scheduled
+// now, before this one finishes; it still waits in pdl_wait() for this kernel's data.
+__device__ __forceinline__ void pdl_release() { asm volatile("griddepcontrol.launch_dependents;"); }
 
 // Index checks of the checked build (compiled with DD_CHECK_BOUNDS). Written as
 // `if (DD_IN_BOUNDS(i < n)) access;`: a false condition records DD_ERR_BOUNDS and

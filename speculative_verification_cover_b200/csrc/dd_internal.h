@@ -55,7 +55,8 @@ struct AttnWorkspace {
 };
 AttnWorkspace attn_workspace_layout(int B, int L, int Hq, int Hkv, int d);
 
-cudaError_t launch_attention(const AttnArgs& a, cudaStream_t stream);
+// prep_done (may be null) is recorded on the stream right after the mask preparation.
+cudaError_t launch_attention(const AttnArgs& a, cudaStream_t stream, cudaEvent_t prep_done);
 
 // Launch `kernel` so that it may start while the previous kernel on `stream` is still
 // finishing (programmatic stream serialization); the kernel calls pdl_wait() before

@@ -29,7 +29,8 @@ DD_MASK_TOKEN = -1
 
 # Every symbol include/dd.h declares.
 EXPORTED = (
-    "dd_dualview_attention", "dd_dualview_attention_ex", "dd_dualview_attention_workspace_size", "dd_verify_logits",
+    "dd_dualview_attention", "dd_dualview_attention_ex", "dd_dualview_attention_ex2",
+    "dd_dualview_attention_workspace_size", "dd_verify_logits",
     "dd_verify_logits_workspace_size", "dd_verify_logits_static",
     "dd_coupled_gumbel", "dd_select_seeds", "dd_select_seeds_ex", "dd_decide",
     "dd_status_string",
@@ -82,6 +83,8 @@ def lib():
     L.dd_dualview_attention.restype = I
     L.dd_dualview_attention_ex.argtypes = [P] * 8 + [I] * 5 + [F, I, I, I, F] + [P] * 5 + [SZ, P]
     L.dd_dualview_attention_ex.restype = I
+    L.dd_dualview_attention_ex2.argtypes = [P] * 8 + [I] * 5 + [F, I, I, I, F] + [P] * 5 + [SZ, P, P]
+    L.dd_dualview_attention_ex2.restype = I
     L.dd_dualview_attention_workspace_size.argtypes = [I] * 5
     L.dd_dualview_attention_workspace_size.restype = SZ
     L.dd_verify_logits.argtypes = [P, P, I, I, I, I, I64, I, F, U64, U64,
@@ -205,18 +208,26 @@ def dd_dualview_attention(q, k_cur, v_cur, k_prev, v_prev, is_seed, is_masked, i
 def dd_dualview_attention_ex(q, k_cur, v_cur, k_prev, v_prev, is_seed, is_masked, is_new,
                              out, lse, d_in=None, d_out=None, workspace=None, q_begin=0,
                              accumulate_stats=False, stats_weight=1.0, softmax_scale=0.0,
-                             stream=None):
+                             stream=None, prep_done=None):
     """One layer of a multi-layer pass with a prefix cache: query rows from q_begin on,
-    this layer's d_in / d_out weighted by stats_weight (see include/dd.h)."""
+    this layer's d_in / d_out weighted by stats_weight (see include/dd.h). prep_done: a
+    torch.cuda.Event recorded right after the mask preparation (dd_dualview_attention_ex2)."""
     B, L, Hq, d = q.shape
     Hkv = k_cur.shape[2]
     nbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
-    st = lib().dd_dualview_attention_ex(
-        _ptr(q), _ptr(k_cur), _ptr(v_cur), _ptr(k_prev), _ptr(v_prev), _ptr(is_seed),
-        _ptr(is_masked), _ptr(is_new), B, L, Hq, Hkv, d, float(softmax_scale), _dtype_code(q),
-        int(q_begin), int(bool(accumulate_stats)), float(stats_weight), _ptr(out), _ptr(lse),
-        _ptr(d_in), _ptr(d_out), _ptr(workspace), nbytes, _stream(stream))
-    _check("dd_dualview_attention_ex", st)
+    args = (_ptr(q), _ptr(k_cur), _ptr(v_cur), _ptr(k_prev), _ptr(v_prev), _ptr(is_seed),
+            _ptr(is_masked), _ptr(is_new), B, L, Hq, Hkv, d, float(softmax_scale), _dtype_code(q),
+            int(q_begin), int(bool(accumulate_stats)), float(stats_weight), _ptr(out), _ptr(lse),
+            _ptr(d_in), _ptr(d_out), _ptr(workspace), nbytes)
+    if prep_done is None:
+        st = lib().dd_dualview_attention_ex(*args, _stream(stream))
+        _check("dd_dualview_attention_ex", st)
+    else:
+        if not prep_done.cuda_event:
+            raise ValueError("prep_done has no CUDA event yet: record it once first")
+        st = lib().dd_dualview_attention_ex2(*args, ctypes.c_void_p(prep_done.cuda_event),
+                                             _stream(stream))
+        _check("dd_dualview_attention_ex2", st)
 
 
 def dd_verify_logits_workspace_size(B, R, V, dtype) -> int:

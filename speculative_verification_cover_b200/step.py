@@ -58,6 +58,9 @@ class VerifyStep:
         self.accepted = torch.empty(B, dtype=torch.uint8, device=dev)
         self.graphs = None
         self.side = None
+        # recorded by the attention call right after its mask preparation (forked())
+        self.prep_done = torch.cuda.Event()
+        self.prep_done.record()  # creates the event
 
     @property
     def n_layers(self):
@@ -68,14 +71,15 @@ class VerifyStep:
         return KERNELS_PER_LAYER * self.n_layers + 4
 
     # --- the four calls
-    def attention(self):
+    def attention(self, prep_done=None):
         x, n = self.x, self.n_layers
         for li, y in enumerate([x] + self.extra_layers):
             dd.dd_dualview_attention_ex(
                 y["q"], y["k_cur"], y["v_cur"], y["k_prev"] if self.use_seeds else None,
                 y["v_prev"] if self.use_seeds else None, x["is_seed"] if self.use_seeds else None,
                 x["is_masked"], x["is_new"], self.out, self.lse, self.d_in, self.d_out, self.ws,
-                q_begin=self.q_begin, accumulate_stats=li > 0, stats_weight=1.0 / n)
+                q_begin=self.q_begin, accumulate_stats=li > 0, stats_weight=1.0 / n,
+                prep_done=prep_done if li == 0 else None)
 
     def verify(self):
         s = self.spec
@@ -104,19 +108,22 @@ class VerifyStep:
         self.select_and_decide()
 
     def forked(self):
-        """The same step on two streams. The vocabulary pass and then the decisions (they
-        read only its statistics) run on a side stream; the attention call runs on the
-        main stream, issued first so that its kernels take SMs ahead of the vocabulary
-        pass. Seed selection needs both, so it waits for the vocabulary pass's event
-        and runs beside the decisions. The attention kernels leave SMs idle at small
-        shapes and the vocabulary pass fills them."""
+        """The same step on two streams. The attention call runs on the main stream; the
+        vocabulary pass and then the decisions (they read only its statistics) run on a
+        side stream that starts once the attention's mask preparation is done: by then
+        the first attention pass holds its SMs (the preparation releases it early), and
+        the vocabulary pass, whose CTAs take chunks of work as they become free, fills
+        every other SM and then the pass's SMs as they empty. Started together instead,
+        the vocabulary pass would take every SM and the attention would wait for it.
+        Seed selection needs both, so it waits for the vocabulary pass's event and runs
+        beside the decisions."""
         main = torch.cuda.current_stream()
         if self.side is None:
             self.side = torch.cuda.Stream(device=main.device)
             self.verified = torch.cuda.Event()
-        self.side.wait_stream(main)
-        self.attention()
+        self.attention(prep_done=self.prep_done)
         with torch.cuda.stream(self.side):
+            self.side.wait_event(self.prep_done)
             self.verify()
             self.verified.record(self.side)
             self.decide()

@@ -165,6 +165,13 @@ def test_attention_ex_validation(lib):
     assert ex(weight=float("nan")) == dd.DD_ERR_INVALID_ARG
     assert ex(weight=float("inf")) == dd.DD_ERR_INVALID_ARG
     assert ex(L=0) == dd.DD_ERR_INVALID_ARG
+    # the variant with a scheduling event validates the same way, before it records anything
+    def ex2(q_begin=0, ws=None):
+        return lib.dd_dualview_attention_ex2(FAKE, FAKE, FAKE, None, None, None, None, None, 1, 8,
+                                             2, 2, 64, 0.0, 1, q_begin, 0, 1.0, FAKE, FAKE,
+                                             None, None, ws, 0, FAKE, None)
+    assert ex2(q_begin=8) == dd.DD_ERR_INVALID_ARG
+    assert ex2() == dd.DD_ERR_INVALID_ARG                   # no workspace
 
 
 def test_select_ex_and_decide_extension_validation(lib):
