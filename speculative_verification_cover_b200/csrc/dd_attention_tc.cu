@@ -161,8 +161,6 @@ attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     }
     uint32_t* neww = reinterpret_cast<uint32_t*>(smem + Lay::kNew);
     const int W = (L + 31) / 32;
-    for (int w = lane; w < W; w += 32) neww[w] = p.newbits[(int64_t)b * W + w];
-    __syncwarp();
     // K(j) may reuse its stage once QK(j - kSK) is done, V(j) once PV(j - kSV) is.
     auto issue_k = [&](int j) -> bool {
       const int s = j % kSK;
@@ -203,6 +201,8 @@ attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       return true;
     };
     // the order the MMA issuer consumes them: K0, K1, V0, K2, V1, K3, V2, ...
+    // The newly-written flags (for V's statistics columns) are read from global
+    // memory after the first K copies are on their way, not before.
     int nk = 0, nv = 0;
     bool ok = issue_k(0);
     if (ok) nk = 1;
@@ -210,6 +210,10 @@ attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       if (j + 1 < T) {
         if (!(ok = issue_k(j + 1))) break;
         nk = j + 2;
+      }
+      if (j == 0) {
+        for (int w = lane; w < W; w += 32) neww[w] = p.newbits[(int64_t)b * W + w];
+        __syncwarp();
       }
       if (!(ok = issue_v(j))) break;
       nv = j + 1;
@@ -287,6 +291,18 @@ attn_p1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     // rank among the sequence's masked rows (-1: not masked or no pass 2)
     const int rank = (p.q_m != nullptr && i < L) ? p.mrank[(int64_t)b * L + i] : -1;
     const float c2 = p.scale_log2;
+    if (seed_row) {
+      // the epilogue's diagonal term reads this row of q, k_cur and v_cur: bring them
+      // into L2 while the tiles stream
+      const int64_t qoff = (((int64_t)b * L + i) * p.Hq + h) * D;
+      const int64_t koff = (((int64_t)b * L + i) * p.Hkv + g) * D;
+#pragma unroll
+      for (int c = 0; c < D * 2; c += 128) {
+        prefetch_l2(reinterpret_cast<const char*>(p.q + qoff) + c);
+        prefetch_l2(reinterpret_cast<const char*>(p.k_cur + koff) + c);
+        prefetch_l2(reinterpret_cast<const char*>(p.v_cur + koff) + c);
+      }
+    }
     float m = -INFINITY;
     bool ok = true;
     for (int j = 0; j < T; ++j) {
