@@ -72,11 +72,16 @@ select_seeds_kernel(const float* __restrict__ entropy, int R, int pos_offset,
   for (int i = threadIdx.x; i < L; i += blockDim.x) {
     const int64_t bi = (int64_t)b * L + i;
     const int r = i - pos_offset;
+    const bool has_row = r >= 0 && r < R;
+    // all four loads at once (one memory round trip); positions without a row read
+    // row 0 (entropy may be NULL only when R = 0)
+    const uint8_t el = eligible[bi];
+    const float u = R > 0 ? entropy[(int64_t)b * R + (has_row ? r : 0)] : 0.f;
+    const float di = d_in[bi], dout = d_out[bi];
     float s = -INFINITY;
     uint32_t key = 0u;
-    if (eligible[bi] && r >= 0 && r < R) {
-      const float u = entropy[(int64_t)b * R + r];
-      s = u * (1.f + d_in[bi]) / (1.f + d_out[bi]);
+    if (el && has_row) {
+      s = u * (1.f + di) / (1.f + dout);
       if (s >= min_score) {  // the adaptive set: only scores reaching the floor compete
         key = orderable(s);
         ++my_cand;

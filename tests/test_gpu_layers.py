@@ -105,3 +105,39 @@ def test_workload_stacks(spec, n_layers, heads):
     torch.cuda.synchronize()
     assert torch.equal(o1[0][:, q_begin:], full[:, q_begin:])
     assert torch.equal(l1[0][:, :, q_begin:], lse[:, :, q_begin:])
+
+
+@pytest.mark.parametrize("spec", [W.LLADA8B_L512, W.TINY_F32], ids=lambda s: s.name)
+def test_prep_done_event_leaves_the_outputs_unchanged(spec):
+    """dd_dualview_attention_ex2 records the caller's event after the mask preparation:
+    a stream that waits on it runs beside the rest of the call, and the call's outputs are
+    bit-identical to dd_dualview_attention_ex's."""
+    x = W.make_inputs(spec, "cuda", with_logits=False)
+    B, L, Hq = spec.B, spec.L, spec.Hq
+    ws = torch.empty(dd.dd_dualview_attention_workspace_size(B, L, Hq, spec.Hkv, spec.d),
+                     dtype=torch.uint8, device="cuda")
+
+    def run(prep_done=None):
+        out = torch.empty_like(x["q"])
+        lse = torch.empty(B, Hq, L, device="cuda")
+        d_in, d_out = torch.empty(B, L, device="cuda"), torch.empty(B, L, device="cuda")
+        dd.dd_dualview_attention_ex(x["q"], x["k_cur"], x["v_cur"], x["k_prev"], x["v_prev"],
+                                    x["is_seed"], x["is_masked"], x["is_new"], out, lse, d_in,
+                                    d_out, ws, prep_done=prep_done)
+        return out, lse, d_in, d_out
+
+    ref = run()
+    torch.cuda.synchronize()
+    ev = torch.cuda.Event()
+    ev.record()  # creates the event
+    side = torch.cuda.Stream()
+    flag = torch.zeros(1, device="cuda")
+    got = run(prep_done=ev)
+    with torch.cuda.stream(side):
+        side.wait_event(ev)
+        flag.fill_(1.0)  # runs once the preparation is done
+    torch.cuda.synchronize()
+    assert dd.dd_get_device_error() == dd.DD_OK
+    assert ev.query() and float(flag) == 1.0
+    for a, b in zip(ref, got):
+        assert torch.equal(a, b)
