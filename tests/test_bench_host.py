@@ -74,3 +74,35 @@ def test_oracle_near_tie_counts_on_a_small_sample():
     bench.oracle_step(x, spec, 0, near=counts)
     assert counts["rows"] == spec.R and "seed_boundary_near" in counts
     assert np.isscalar(counts["near_decisions"])
+
+
+def test_reference_arm_prints_the_contract_line():
+    """`bench.py --impl reference` (the fp64 oracle on the host cores) prints one JSON line
+    with the contract's keys, on the arm's own config, and exits 0 without a GPU."""
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    res = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference",
+                          "--workload", W.TINY_F32.name, "--steps", "2", "--warmup", "1"],
+                         capture_output=True, text=True, timeout=300, cwd=root)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [ln for ln in res.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC
+    assert d["value"] > 0 and d["unit"] == "steps/s" and d["higher_is_better"] is True
+    assert d["steps"] == 2 and d["warmup"] == 1 and d["n_gpus"] == 1
+    assert d["config"]["workload"] == W.TINY_F32.name
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": "steps/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+
+
+def test_kernel_count_per_step():
+    """gpu_launches counts our kernels: per attention layer the preparation, the two passes
+    and the head reduction; then the vocabulary stream and merge, selection, decisions."""
+    from speculative_verification_cover_b200 import step
+    assert step.KERNELS_PER_STEP == 8
