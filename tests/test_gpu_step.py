@@ -95,3 +95,33 @@ def test_one_graph_step_matches_the_serial_calls(spec):
     got += [step.out, step.d_in, step.d_out]
     for a, b in zip(ref, got):
         assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("prefix_cache", [False, True])
+def test_multilayer_graph_step_matches_the_serial_calls(prefix_cache):
+    """A three-layer step as one CUDA graph (the vocabulary pass starting once the first
+    layer's mask preparation is done) gives bit-identical results to the calls made in
+    order; with the prefix cache, each layer computes the rows after the prompt only."""
+    from speculative_verification_cover_b200.step import VerifyStep
+    spec = W.LLADA8B_L512
+    x = W.make_inputs(spec, "cuda")
+    extra = W.layer_operands(spec, "cuda", seed=11, n_layers=2)
+    step = VerifyStep(spec, x, extra_layers=extra, prefix_cache=prefix_cache)
+    step.choose_initial_seeds()
+    step()  # serial, eager
+    torch.cuda.synchronize()
+    names = ("lse_t", "entropy_t", "kl_dt", "argmax_t", "sample_t")
+    ref = [t.clone() for t in step.result_tensors()] + [getattr(step.stats, n).clone() for n in names]
+    ref += [step.d_in.clone(), step.d_out.clone(), step.score.clone()]
+    step.capture()
+    for t in step.result_tensors():
+        t.fill_(0x55)
+    step.d_in.fill_(7.0)
+    step.replay()
+    torch.cuda.synchronize()
+    assert dd.dd_get_device_error() == dd.DD_OK
+    got = [t for t in step.result_tensors()] + [getattr(step.stats, n) for n in names]
+    got += [step.d_in, step.d_out, step.score]
+    for a, b in zip(ref, got):
+        assert torch.equal(a, b)
+    step.graphs = None
