@@ -60,7 +60,8 @@ class VerifyStep:
         self.side = None
         # recorded by the attention call right after its mask preparation (forked())
         self.prep_done = torch.cuda.Event()
-        self.prep_done.record()  # creates the event
+        with torch.cuda.device(dev):
+            self.prep_done.record()  # creates the event on the inputs' device
 
     @property
     def n_layers(self):
